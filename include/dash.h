@@ -299,8 +299,10 @@ int dash_decode_paged(const dash_problem* p, const int32_t* cache_lens, const in
  * about 6 MB (the 8-sequence, 2-KV-head, 131072-token cache case about
  * 4.7 MB); a problem whose scratch exceeded 8 MiB would return
  * DASH_ERR_WORKSPACE.
- * The first call on a device looks up that device's address of the array
- * (with the device current); make that first call before any stream capture.
+ * Every call looks up the current device's address of the array (with that
+ * device current), so a device reset between calls leaves nothing stale; the
+ * first call on a device also loads the library's device code there, so make
+ * that first call before any stream capture.
  * All calls on a device share the one array and it keeps the last call's
  * contents (nothing in it needs to start at zero), so calls that overlap on
  * the GPU -- concurrent streams, or threads using the same device -- race
@@ -329,6 +331,18 @@ int dash_get_error(void* stream);
  * or hangs.  Returns DASH_ERR_CUDA if the launch fails, else DASH_OK.
  */
 int dash_selftest_wait_timeout(void* stream);
+
+/*
+ * Accuracy self-test (no counterpart in the pages): y[i] = the attention
+ * kernel's FMA-pipe evaluation of 2^x[i] (a Cody-Waite split x = n + f,
+ * |f| <= 1/2, and a degree-3 polynomial for 2^f fitted for minimum maximum
+ * relative error, 7.5e-5), which computes part of stage 2's softmax
+ * exponentials.  Inputs below -125 are clamped to -125 (so -inf gives
+ * about 2^-125, not 0).  x and y: device float [n], 4-byte aligned.
+ * Returns DASH_ERR_INVALID_ARG for n < 0 or NULL pointers with n > 0,
+ * DASH_ERR_CUDA if the launch fails, else DASH_OK.
+ */
+int dash_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
 
 #ifdef __cplusplus
 }

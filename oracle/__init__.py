@@ -33,4 +33,6 @@ from .dash_oracle import (  # noqa: F401
     decode,
     decode_varlen,
     decode_paged,
+    decode_attend,
+    gather_pages,
 )

@@ -79,6 +79,11 @@ What pins each function (``tests/test_oracle.py``):
   cache rebuilds ``chunk_summary`` of the whole cache; rows of sequences not
   at a boundary are left as they were; the paged form equals the contiguous
   one through an identity table.
+* ``decode_attend`` (stage 2 of a decode step on given routing): with every
+  chunk active and w = 1 it is torch's SDPA of each query against its first
+  L keys; on ``decode``'s own routing it returns ``decode``'s output; with one
+  routed chunk it is a softmax over that chunk (bias sigma ln w) and the
+  query's own causal chunk.
 * ``decode_paged``: an identity page table over a pool that is the caches
   cut into pages gives ``decode_varlen``; permuting the pool's pages together
   with the table, and rewriting pages no table entry of a sequence's own
@@ -428,6 +433,23 @@ def decode_paged(q, Kpool, Vpool, Kbar, lens, page_table, alpha, gamma, sigma, B
     n_pages, hkv, Bp, d = Kpool.shape
     if Bp != B:
         raise ValueError("a page holds one chunk of B tokens")
+    Kc, Vc = gather_pages(Kpool, Vpool, lens, page_table, B)
+    return decode_varlen(q, Kc, Vc, Kbar, lens, alpha, gamma, sigma, B, near_tol)
+
+
+def gather_pages(Kpool, Vpool, lens, page_table, B):
+    """Contiguous caches [b, H_kv, max_pages * B, d] from one-chunk pages.
+
+    Chunk c of sequence bi (for c below ceil(lens[bi] / B)) is copied from
+    page page_table[bi, c]; the rest stays zero.  A page id outside the pool
+    raises ValueError.
+    """
+    Kpool, Vpool = _f64(Kpool), _f64(Vpool)
+    table = np.asarray(page_table)
+    b = table.shape[0]
+    n_pages, hkv, Bp, d = Kpool.shape
+    if Bp != B:
+        raise ValueError("a page holds one chunk of B tokens")
     cap = table.shape[1] * B
     Kc = np.zeros((b, hkv, cap, d))
     Vc = np.zeros((b, hkv, cap, d))
@@ -438,7 +460,42 @@ def decode_paged(q, Kpool, Vpool, Kbar, lens, page_table, alpha, gamma, sigma, B
                 raise ValueError(f"page id {pg} outside [0, {n_pages})")
             Kc[bi, :, c * B:(c + 1) * B] = Kpool[pg]
             Vc[bi, :, c * B:(c + 1) * B] = Vpool[pg]
-    return decode_varlen(q, Kc, Vc, Kbar, lens, alpha, gamma, sigma, B, near_tol)
+    return Kc, Vc
+
+
+def decode_attend(q, Kc, Vc, w, mask, lens, sigma, B):
+    """Stage 2 alone of a decode step, on given routing weights and mask.
+
+    The prior-induced sparse softmax of gist.science summary "Fase 2" for
+    the single query of each sequence (position lens[bi] - 1 of its cache):
+    the routed chunks of ``mask`` below the query's own chunk with bias
+    sigma * ln w, and the query's own chunk (causal) with bias 0.  This is
+    the second half of ``decode`` with its routing replaced by the caller's,
+    so a decode kernel's attention output can be compared on the kernel's
+    own routing.
+
+    q: [b, H_q, d]; Kc, Vc: [b, H_kv, >= lens, d]; w: [b, H_kv, n_c];
+    mask: [b, H_kv, n_w]; lens: per-sequence cache lengths (None: all
+    Kc.shape[2]).  Returns (o [b, H_q, d], lse [b, H_q]).
+    """
+    q, Kc, Vc, w = _f64(q), _f64(Kc), _f64(Vc), _f64(w)
+    b, hq, d = q.shape
+    hkv, cap = Kc.shape[1], Kc.shape[2]
+    G = hq // hkv
+    active = unpack_mask(np.asarray(mask), w.shape[-1])
+    lens = [cap] * b if lens is None else [int(L) for L in lens]
+    o = np.zeros((b, hq, d))
+    lse = np.zeros((b, hq))
+    for bi in range(b):
+        L = lens[bi]
+        if not 1 <= L <= cap:
+            raise ValueError(f"cache length {L} outside [1, {cap}]")
+        for g in range(hkv):
+            og, lg = _attend(q[bi, g * G:(g + 1) * G], Kc[bi, g, :L], Vc[bi, g, :L], w[bi, g],
+                             active[bi, g], L - 1, B, sigma)
+            o[bi, g * G:(g + 1) * G] = og
+            lse[bi, g * G:(g + 1) * G] = lg
+    return o, lse
 
 
 def summarize_append(K, qbar, Kbar, lens, B, page_table=None):

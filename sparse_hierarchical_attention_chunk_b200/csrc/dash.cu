@@ -10,8 +10,6 @@
 #include <stdint.h>
 #include <string.h>
 
-#include <mutex>
-
 #include "dash.h"
 #include "dash_common.cuh"
 #include "tmap.cuh"
@@ -424,6 +422,18 @@ __global__ void selftest_wait_kernel() {
   if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, nullptr);
 }
 
+// Evaluates the attention kernel's FMA-pipe 2^x (exp2_poly2) on n inputs, so
+// that its error can be measured against 2^x itself.
+__global__ void selftest_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x1 = i + 1 < n ? x[i + 1] : 0.f;
+  float e0, e1;
+  exp2_poly2(f2_pack(x[i], x1), e0, e1);
+  y[i] = e0;
+  if (i + 1 < n) y[i + 1] = e1;
+}
+
 }  // namespace dash
 
 namespace {
@@ -431,25 +441,17 @@ namespace {
 constexpr size_t kDecodeStaticScratchBytes = size_t(8) << 20;   // 8 MiB
 static __device__ __align__(256) uint8_t g_decode_static_scratch[kDecodeStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_scratch_mu;
-void* g_static_scratch_ptr[kMaxDevices] = {};
-
 // Device address of the static scratch on the current device.  In host code
-// the array's name is only a stand-in, so the real address is looked up once
-// per device (with that device current) and cached.
+// the array's name is only a stand-in, so the address is looked up with the
+// device current.  The lookup is repeated on every call (after the first call
+// on a device has loaded the library's device code it is a table lookup), so
+// a device reset or a re-created primary context never leaves a stale
+// address behind.
 int static_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaErrorInvalidDevice);
-  if (dev < 0 || dev >= kMaxDevices) return DASH_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-  if (!g_static_scratch_ptr[dev]) {
-    void* ptr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&ptr, g_decode_static_scratch);
-    if (e != cudaSuccess || !ptr) return cuda_status(e == cudaSuccess ? cudaErrorUnknown : e);
-    g_static_scratch_ptr[dev] = ptr;
-  }
-  *out = g_static_scratch_ptr[dev];
+  void* ptr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&ptr, g_decode_static_scratch);
+  if (e != cudaSuccess || !ptr) return cuda_status(e == cudaSuccess ? cudaErrorUnknown : e);
+  *out = ptr;
   return DASH_OK;
 }
 
@@ -489,6 +491,14 @@ int dash_decode_noalloc(const dash_problem* p, const void* q, const void* Kcache
 
 int dash_selftest_wait_timeout(void* stream) {
   dash::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return cuda_status(cudaGetLastError());
+}
+
+int dash_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return DASH_ERR_INVALID_ARG;
+  if (n == 0) return DASH_OK;
+  const int pairs = (n + 1) / 2;
+  dash::selftest_exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return cuda_status(cudaGetLastError());
 }
 

@@ -1029,13 +1029,12 @@ inline int run_decode(int batch, int n_q, int n_kv, int L, int D, int chunk, flo
   const uint64_t str[1] = {(uint64_t)D * 2};
   const uint32_t box[2] = {64, (uint32_t)chunk};
   if (!make_tmap(&tk, Kc, 2, dims, str, box) || !make_tmap(&tv, Vc, 2, dims, str, box)) return 3;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0, v = 148;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) v = 148;
-    sms = v;
-  }
+  // SM count of the current device, read on every call (a host-side lookup):
+  // the split grid is sized for the device the call runs on
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return 3;
   const int n_ctas = decode_split_ctas(n_bg, c_q, sms);
   DecodeSplitParams prm;
   prm.q = q;

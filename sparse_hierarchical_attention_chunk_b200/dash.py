@@ -31,7 +31,8 @@ DASH_BF16 = 1
 EXPORTED = ("dash_status_str", "dash_version", "dash_summarize", "dash_route", "dash_attn_fwd",
             "dash_workspace_bytes", "dash_decode", "dash_decode_varlen", "dash_decode_paged",
             "dash_get_error", "dash_decode_noalloc", "dash_summarize_append", "dash_route_topk",
-            "dash_attn_bwd", "dash_route_bwd", "dash_summarize_bwd", "dash_selftest_wait_timeout")
+            "dash_attn_bwd", "dash_route_bwd", "dash_summarize_bwd", "dash_selftest_wait_timeout",
+            "dash_selftest_exp2_poly")
 
 
 class DashError(RuntimeError):
@@ -98,6 +99,8 @@ def lib():
                                         ctypes.c_size_t, vp]
         L.dash_selftest_wait_timeout.restype = i32
         L.dash_selftest_wait_timeout.argtypes = [vp]
+        L.dash_selftest_exp2_poly.restype = i32
+        L.dash_selftest_exp2_poly.argtypes = [vp, vp, i32, vp]
         L.dash_get_error.restype = i32
         L.dash_get_error.argtypes = [vp]
         L.dash_decode_noalloc.restype = i32
@@ -388,6 +391,14 @@ def dash_selftest_wait_timeout(stream=None):
     """Run the library's bounded-wait timeout path once (about 2 s); the next
     dash_get_error returns DASH_ERR_TIMEOUT."""
     _raise("dash_selftest_wait_timeout", lib().dash_selftest_wait_timeout(_stream(stream)))
+
+
+def dash_selftest_exp2_poly(x, y, stream=None):
+    """y = the attention kernel's FMA-pipe 2^x on a float32 device tensor x."""
+    _check(x, "x", (x.numel(),), torch.float32)
+    _check(y, "y", (x.numel(),), torch.float32)
+    _raise("dash_selftest_exp2_poly",
+           lib().dash_selftest_exp2_poly(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)))
 
 
 def dash_get_error(stream=None):

@@ -22,7 +22,7 @@ def L():
 def _declared():
     text = open(os.path.join(ROOT, "include", "dash.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(dash_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(dash_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_binding_names():

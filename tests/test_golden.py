@@ -1,4 +1,9 @@
-"""The oracle against its stored regression fixture (see tests/golden/README.md)."""
+"""The oracle against its stored regression fixture.
+
+The pages print no worked numeric example, so the fixture is not a pin: it
+was written by tests/golden/make_golden.py, which calls only the oracle and
+the seeded input generator, and it guards the oracle against unintended
+changes between commits."""
 
 import json
 import os

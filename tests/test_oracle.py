@@ -383,6 +383,57 @@ def test_decode_equals_last_prefill_row(L):
     np.testing.assert_allclose(wd, w[:, :, 0, :wd.shape[-1]], atol=0)
 
 
+def test_decode_attend_dense_is_sdpa_of_the_last_row():
+    # every chunk active with w = 1: the prior is uniform over the causal
+    # prefix for any sigma, so each sequence's output is torch's SDPA of its
+    # query against its first L keys
+    rng = np.random.default_rng(25)
+    b, hq, hkv, d, B, cap = 3, 4, 2, 16, 16, 160
+    lens = [160, 1, 77]
+    q = rng.normal(size=(b, hq, d))
+    K = rng.normal(size=(b, hkv, cap, d))
+    V = rng.normal(size=(b, hkv, cap, d))
+    n_c = cap // B
+    w = np.ones((b, hkv, n_c))
+    mask = oracle.pack_mask(w > 0)
+    o, lse = oracle.decode_attend(q, K, V, w, mask, lens, 0.9, B)
+    for bi, L in enumerate(lens):
+        tq = torch.from_numpy(q[bi][None, :, None, :])
+        tk, tv = (torch.from_numpy(a[bi][None, :, :L]) for a in (K, V))
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, enable_gqa=True)
+        np.testing.assert_allclose(o[bi], ref[0, :, 0].numpy(), atol=1e-12)
+        s = np.einsum("hd,hkd->hk", q[bi], np.repeat(K[bi, :, :L], 2, axis=0)) / math.sqrt(d)
+        np.testing.assert_allclose(lse[bi], torch.logsumexp(torch.from_numpy(s), dim=1).numpy(),
+                                   atol=1e-12)
+
+
+def test_decode_attend_on_decode_routing_is_decode_and_prefill_row():
+    # fed the routing that decode computes, stage 2 alone gives decode's output,
+    # i.e. the last prefill row (itself pinned to dense SDPA and the variational
+    # form); fed a different routing it follows that routing instead
+    rng = np.random.default_rng(26)
+    b, hq, hkv, d, B, L = 2, 4, 2, 16, 16, 150
+    Q = rng.normal(size=(b, hq, L, d))
+    K = rng.normal(size=(b, hkv, L, d))
+    V = rng.normal(size=(b, hkv, L, d))
+    Kbar = oracle.chunk_summary(K, rng.normal(size=(hkv, d)) * 0.1, B)
+    o, lse, w, mask, _ = oracle.decode(Q[:, :, L - 1], K, V, Kbar, L, 1.5, 0.9, 0.7, B)
+    o2, lse2 = oracle.decode_attend(Q[:, :, L - 1], K, V, w, mask, None, 0.7, B)
+    np.testing.assert_array_equal(o2, o)
+    np.testing.assert_array_equal(lse2, lse)
+    # one routed chunk (chunk 2, weight 0.3) plus the query's own chunk 9 (keys 144..149)
+    w1 = np.zeros_like(w)
+    w1[..., 2] = 0.3
+    o3, _ = oracle.decode_attend(Q[:, :, L - 1], K, V, w1, oracle.pack_mask(w1 > 0), None, 2.0, B)
+    keys = list(range(32, 48)) + list(range(144, 150))
+    for bi in range(b):
+        for h in range(hq):
+            s = K[bi, h // 2, keys] @ Q[bi, h, L - 1] / math.sqrt(d)
+            s[:16] += 2.0 * math.log(0.3)
+            p = np.exp(s - s.max())
+            np.testing.assert_allclose(o3[bi, h], (p / p.sum()) @ V[bi, h // 2, keys], atol=1e-12)
+
+
 def _varlen_case(seed, b=3, hq=4, hkv=2, d=16, B=16, L_max=200):
     rng = np.random.default_rng(seed)
     q = rng.normal(size=(b, hq, d))

@@ -232,26 +232,29 @@ def test_end_to_end_tiny_f32(zero_qbar):
 
 
 def test_end_to_end_bf16():
+    # the GPU chain (summaries -> routing -> attention, one dash.prefill call);
+    # every output is compared, each stage against the oracle run on the
+    # GPU's own upstream result (a bf16 summary one ulp away from the
+    # oracle's moves a logit by ~1e-3, which would otherwise decide mask
+    # bits near the threshold differently)
     wl = MED["g16_d128_b64_nc37"]
     inp = synth.make_prefill(wl, seed=11)
     p = dash.problem_for(wl)
     out = dash.prefill(p, inp["Q"].cuda(), inp["K"].cuda(), inp["V"].cuda(), inp["qbar"].cuda())
     torch.cuda.synchronize()
-    # the oracle's chain with its summaries stored in bf16, as the kernels store them
-    kb = oracle_kbar(inp["K"], inp["qbar"], wl.chunk, torch.bfloat16)
-    wr, mr, near = oracle.route(inp["Q"], kb, wl.alpha, wl.gamma, wl.chunk, near_tol=2e-2)
+    ref_kb = oracle.chunk_summary(inp["K"], inp["qbar"], wl.chunk)
+    kb = np64(out["Kbar"])
+    assert np.all(np.abs(kb - ref_kb) <= 2.0 ** -8 * np.abs(ref_kb) + 1e-6)
+    wr, mr, near = oracle.route(inp["Q"], out["Kbar"].cpu(), wl.alpha, wl.gamma, wl.chunk)
     mg = mask_from_dev(out["mask"])
-    # bf16 storage of the summaries may move a logit by ~1e-3: flips are
-    # allowed only where some head's score lies within 2e-2 of its threshold
     n_diff, n_bad = compare_masks(mg, mr, near, wl.n_chunks)
+    print(f"near-threshold mask flips: {n_diff}")
     assert n_bad == 0
-    rows_same = np.all(mg == mr, axis=-1)                      # [b, h_kv, N]
-    Or, lr = oracle.attn_fwd(inp["Q"], inp["K"], inp["V"], wr, mr, wl.sigma, wl.chunk)
-    G = wl.group
-    keep = np.repeat(rows_same, G, axis=1)[..., None]
-    err = np.where(keep, np.abs(np64(out["O"]) - Or), 0.0)
-    assert err.max() <= TOL_O_BF16
-    assert rows_same.mean() > 0.9
+    wg = np64(out["w"])
+    assert np.abs(wg - wr).max() <= TOL_W
+    Or, lr = oracle.attn_fwd(inp["Q"], inp["K"], inp["V"], wg, mg, wl.sigma, wl.chunk)
+    assert np.abs(np64(out["O"]) - Or).max() <= TOL_O_BF16
+    assert np.abs(np64(out["lse"]) - lr).max() <= TOL_LSE
 
 
 # ----------------------------------------------------------------------------
@@ -338,35 +341,24 @@ def _decode_case(wl, seed):
     p = dash.problem_for(wl)
     out = dash.decode(p, inp["q"].cuda(), inp["K"].cuda(), inp["V"].cuda(), kb.cuda())
     assert dash.dash_get_error() == dash.DASH_OK
-    o, lse, w, mask, near = oracle.decode(inp["q"], inp["K"], inp["V"], kb, wl.seq, wl.alpha,
-                                          wl.gamma, wl.sigma, wl.chunk)
-    return out, (o, lse, w, mask, near)
+    ref = oracle.decode(inp["q"], inp["K"], inp["V"], kb, wl.seq, wl.alpha, wl.gamma, wl.sigma,
+                        wl.chunk)
+    return out, ref, inp, kb
 
 
 @pytest.mark.parametrize("name", list(DEC))
 def test_decode_matches_oracle(name):
     wl = DEC[name]
-    out, (o, lse, w, mask, near) = _decode_case(wl, seed=12)
-    n_diff, n_bad = compare_masks(mask_from_dev(out["mask"]), mask, near, wl.n_chunks)
-    assert n_bad == 0
+    out, ref, inp, kb = _decode_case(wl, seed=12)
     if name.endswith("_dense"):                    # the case must really be dense
         assert (np64(out["w"])[..., : (wl.seq - 1) // wl.chunk] > 0).all()
-    assert np.abs(np64(out["w"]) - w).max() <= TOL_W
-    if n_diff == 0:
-        assert np.abs(np64(out["o"]) - o).max() <= TOL_O_BF16
-        assert np.abs(np64(out["lse"]) - lse).max() <= TOL_LSE
+    _check_decode(wl, out, ref, inp["q"], inp["K"], inp["V"], None)
 
 
 def test_decode_full_size():
     wl = configs.DECODE_128K
-    out, (o, lse, w, mask, near) = _decode_case(wl, seed=0)
-    n_diff, n_bad = compare_masks(mask_from_dev(out["mask"]), mask, near, wl.n_chunks)
-    assert n_bad == 0
-    assert np.abs(np64(out["w"]) - w).max() <= TOL_W
-    same = np.all(mask_from_dev(out["mask"]) == mask, axis=-1)          # [b, h_kv]
-    keep = np.repeat(same, wl.group, axis=1)[..., None]
-    assert np.where(keep, np.abs(np64(out["o"]) - o), 0).max() <= TOL_O_BF16
-    assert same.mean() > 0.8
+    out, ref, inp, kb = _decode_case(wl, seed=0)
+    _check_decode(wl, out, ref, inp["q"], inp["K"], inp["V"], None)
 
 
 def test_decode_equals_prefill_last_row_on_gpu():
@@ -411,36 +403,46 @@ def _decode_varlen_case(wl, lens, seed):
     assert dash.dash_get_error() == dash.DASH_OK
     ref = oracle.decode_varlen(inp["q"], inp["K"], inp["V"], kb, lens.tolist(), wl.alpha, wl.gamma,
                                wl.sigma, wl.chunk)
-    return out, ref, lens
+    return out, ref, lens, inp
 
 
-def _check_decode(wl, out, ref, min_same=1.0):
+def _check_decode(wl, out, ref, q, Kc, Vc, lens):
+    """Every output of a decode call against the oracle.
+
+    Routing (D0): the mask bit-exact except at chunks where some head's score
+    lies within 1e-4 of its threshold (counted and printed), w within 1e-3.
+    Attention (D1 + D2): o and lse of every (sequence, KV head), against the
+    oracle's stage 2 run on the kernel's own w and mask, so that a legitimate
+    flip at the threshold cannot hide or excuse an attention error.  Where the
+    whole mask of a (sequence, KV head) equals the oracle's, o is also checked
+    against the oracle's own end-to-end result.
+    """
     o, lse, w, mask, near = ref
     gm = mask_from_dev(out["mask"])
     n_diff, n_bad = compare_masks(gm, mask, near, wl.n_chunks)
-    assert n_bad == 0
-    assert np.abs(np64(out["w"]) - w).max() <= TOL_W
-    # outputs of the (b, h_kv) whose active set matches exactly (a chunk at
-    # the threshold may flip, and then its keys legitimately change o)
-    same = np.all(gm == mask, axis=-1)
-    assert same.mean() >= min_same
-    keep = np.repeat(same, wl.group, axis=1)
-    assert np.where(keep[..., None], np.abs(np64(out["o"]) - o), 0).max() <= TOL_O_BF16
-    assert np.where(keep, np.abs(np64(out["lse"]) - lse), 0).max() <= TOL_LSE
+    print(f"near-threshold mask flips: {n_diff}")
+    assert n_bad == 0, f"{n_bad} mask bits differ away from tau ({n_diff} total)"
+    wg = np64(out["w"])
+    assert np.abs(wg - w).max() <= TOL_W
+    o_iso, lse_iso = oracle.decode_attend(q, Kc, Vc, wg, gm, lens, wl.sigma, wl.chunk)
+    assert np.abs(np64(out["o"]) - o_iso).max() <= TOL_O_BF16
+    assert np.abs(np64(out["lse"]) - lse_iso).max() <= TOL_LSE
+    same = np.repeat(np.all(gm == mask, axis=-1), wl.group, axis=1)        # [b, h_q]
+    assert np.where(same[..., None], np.abs(np64(out["o"]) - o), 0).max() <= TOL_O_BF16
 
 
 @pytest.mark.parametrize("name", list(DECV))
 def test_decode_varlen_matches_oracle(name):
     wl, lens = DECV[name]
-    out, ref, _ = _decode_varlen_case(wl, lens, seed=14)
-    _check_decode(wl, out, ref)
+    out, ref, lens, inp = _decode_varlen_case(wl, lens, seed=14)
+    _check_decode(wl, out, ref, inp["q"], inp["K"], inp["V"], lens.tolist())
 
 
 def test_decode_varlen_full_size():
     wl = configs.DECODE_VARLEN_128K
-    out, ref, lens = _decode_varlen_case(wl, None, seed=0)
+    out, ref, lens, inp = _decode_varlen_case(wl, None, seed=0)
     assert lens.min().item() >= wl.seq // 8 and lens.max().item() <= wl.seq
-    _check_decode(wl, out, ref, min_same=0.8)
+    _check_decode(wl, out, ref, inp["q"], inp["K"], inp["V"], lens.tolist())
 
 
 def test_decode_varlen_reads_nothing_past_each_length():
@@ -508,14 +510,15 @@ def _decode_paged_case(wl, lens, seed, extra_pages=7):
     assert dash.dash_get_error() == dash.DASH_OK
     ref = oracle.decode_paged(inp["q"], Kp, Vp, kb, lens.tolist(), table.numpy(), wl.alpha,
                               wl.gamma, wl.sigma, wl.chunk)
-    return out, ref
+    Kc, Vc = oracle.gather_pages(Kp, Vp, lens.tolist(), table.numpy(), wl.chunk)
+    return out, ref, (inp["q"], Kc, Vc, lens.tolist())
 
 
 @pytest.mark.parametrize("name", list(DECV))
 def test_decode_paged_matches_oracle(name):
     wl, lens = DECV[name]
-    out, ref = _decode_paged_case(wl, lens, seed=18)
-    _check_decode(wl, out, ref)
+    out, ref, (q, Kc, Vc, lens) = _decode_paged_case(wl, lens, seed=18)
+    _check_decode(wl, out, ref, q, Kc, Vc, lens)
 
 
 def test_decode_paged_full_size_equals_varlen():
@@ -623,7 +626,7 @@ def test_incremental_decode_loop():
         assert dash.dash_get_error() == dash.DASH_OK
         ref = oracle.decode_varlen(q, inp["K"], inp["V"], kb_ref, lens, wl.alpha, wl.gamma, wl.sigma,
                                    wl.chunk)
-        _check_decode(wl, out, ref)
+        _check_decode(wl, out, ref, q, inp["K"], inp["V"], lens)
         dash.dash_summarize_append(p, dl, K, qbar, kb)
     full = torch.empty_like(kb)
     dash.dash_summarize(p, K, qbar, full)
