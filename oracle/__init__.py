@@ -24,6 +24,7 @@ from .dash_oracle import (  # noqa: F401
     entmax_bisect,
     entmax15_sort,
     chunk_summary,
+    diagonal_summary,
     summarize_append,
     route,
     route_topk,

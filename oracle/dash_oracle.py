@@ -45,6 +45,15 @@ Readings where the pages are silent (each is listed in the design notes):
   ignored.
 * Decode: the new query is position L-1 of an L-token cache that already
   holds its own key/value; it equals row L-1 of prefill on the same data.
+* estimate_diagonal (aiexpert.news article, interface paragraph: a flag for
+  a diagonal correction of the alpha-entmax normalisation; gist.science
+  summary, Fase 2 "Diagonaal Afhandeling": chunks near the diagonal may have
+  no summary): the query's own chunk, whose summary does not exist yet, is
+  given an estimated one -- stage 0's learned-query summary over the keys
+  the query may see (its chunk's start .. i) -- and joins the entmax as one
+  more candidate, so the routed chunks share 1 - w_diag of the mass.  The
+  diagonal branch of stage 2 stays on with weight 1 whatever w_diag is;
+  w_diag is reported in column c_i of w and never sets a mask bit.
 * Top-k routing (the fixed-budget baseline the pages contrast with, NSA and
   InfLLMv2): the coarse score of a chunk is the group mean of the per-head
   softmax of gamma z_bar over the eligible chunks; the k best chunks (equal
@@ -62,12 +71,21 @@ What pins each function (``tests/test_oracle.py``):
   chunk's keys; invariant to permuting keys inside a chunk.
 * ``route``: G = 1 equals one brute-force entmax per row on hand-computed
   logits; w sums to one on rows with eligible chunks; mask = OR of the
-  per-head supports; empty for the first chunk.
+  per-head supports; empty for the first chunk.  With the diagonal
+  candidate: a hand-computed sparsemax case (two candidates, B = 2, the
+  estimate written out key by key); at the last row of a chunk the estimate
+  is the chunk's complete summary, so the weights equal plain routing of the
+  same query one position later; the routed chunks and the diagonal sum to
+  one; rows of the first chunk give the diagonal weight 1; the mask never
+  holds the query's own chunk.
+* ``diagonal_summary``: ``chunk_summary`` of the partial chunk (pinned
+  through the chunk-end case above and the hand-computed case).
 * ``attn_fwd``: all chunks active with sigma = 0 equals dense causal softmax
   attention (torch's fp64 scaled_dot_product_attention); one-hot values
   expose p, which is checked against the variational optimality condition
   of z^T p - KL(p || g); a single active block reduces to a local softmax.
-* ``decode``: equals the last row of prefill on the same data.
+* ``decode``: equals the last row of prefill on the same data (with and
+  without the diagonal candidate).
 * ``decode_varlen``: each sequence equals the last row of prefill on its own
   prefix; equal lengths reduce to ``decode``; nothing past a sequence's
   length (cache rows, summary rows) changes its result.
@@ -240,7 +258,23 @@ def chunk_summary(K, qbar, B, chunk_begin=0, chunk_end=None):
 # Stage 1: entmax chunk routing with GQA averaging
 # ----------------------------------------------------------------------------
 
-def route(Q, Kbar, alpha, gamma, B, positions=None, near_tol=1e-4, return_heads=False):
+def diagonal_summary(K, qbar, B, i):
+    """Estimated summary of the query's own chunk for the query at position i.
+
+    The chunk c_i = floor(i / B) is not complete when its row i is routed, so
+    it has no cached summary (gist.science summary, Fase 2 "Diagonaal
+    Afhandeling": chunks near the diagonal may have no summary).  The
+    estimate is stage 0's learned-query summary taken over the keys the query
+    may see, c_i B .. i: ``chunk_summary`` of that partial chunk.  K: [H_kv, >=
+    i + 1, d] of one sequence; qbar: [H_kv, d].  Returns fp64 [H_kv, d].
+    """
+    c_i = i // B
+    part = _f64(K)[None, :, c_i * B:i + 1, :]
+    return chunk_summary(part, qbar, i + 1 - c_i * B)[0, :, 0, :]
+
+
+def route(Q, Kbar, alpha, gamma, B, positions=None, near_tol=1e-4, return_heads=False,
+          diag=None):
     """Routing weights and active-block mask.
 
     Q: [b, H_q, N, d]; Kbar: [b, H_kv, n_c, d] (n_c = number of chunk rows
@@ -248,6 +282,16 @@ def route(Q, Kbar, alpha, gamma, B, positions=None, near_tol=1e-4, return_heads=
     z[h, c] = Q[b, h, i] . Kbar[b, h_kv, c] for eligible c < floor(i / B);
     p[h] = alpha-entmax(gamma z[h]); w = mean over the G query heads of the
     KV group; mask bit = (w > 0).
+
+    diag = (K [b, H_kv, N, d], qbar [H_kv, d]) turns on estimate_diagonal
+    (aiexpert.news article, interface paragraph: a diagonal correction of the
+    alpha-entmax normalisation): the query's own chunk c_i joins the entmax
+    as one more candidate, with logit z[h, c_i] = Q[b, h, i] .
+    ``diagonal_summary``(i).  Its group-mean weight is written to w[..., c_i];
+    the routed chunks c < c_i then share 1 - w[..., c_i].  The mask keeps
+    only the routed chunks (bit c_i stays clear: the query's own chunk is
+    attended by its own branch in stage 2 whatever its weight).  Rows of the
+    first chunk have the diagonal as their only candidate: w[..., 0] = 1.
 
     Returns (w [b, H_kv, P, n_c] fp64, mask [b, H_kv, P, n_w] uint32,
     near [b, H_kv, P, n_c] bool) where near marks chunks for which some head
@@ -270,18 +314,36 @@ def route(Q, Kbar, alpha, gamma, B, positions=None, near_tol=1e-4, return_heads=
             for c_i in np.unique(chunk_of):
                 sel = np.nonzero(chunk_of == c_i)[0]
                 ne = int(min(c_i, n_c))
-                if ne == 0:
+                with_diag = diag is not None and c_i < n_c
+                if ne == 0 and not with_diag:
                     continue
                 Zq = _take(Q, bi, g * G, (g + 1) * G, pos[sel])          # [G, S, d]
                 z = Zq @ Kb[:ne, :].T                                   # [G, S, ne]
-                p = entmax_bisect(gamma * z, alpha)                     # [G, S, ne]
+                if with_diag:
+                    Kd = _take(diag[0], bi, g, g + 1, np.arange(c_i * B, (c_i + 1) * B))[0]
+                    est = np.stack([diagonal_summary(Kd[None], _f64(diag[1])[g:g + 1], B,
+                                                     int(i) - c_i * B)[0] for i in pos[sel]])
+                    zd = np.einsum("gsd,sd->gs", Zq, est)               # [G, S]
+                    z = np.concatenate([z, zd[..., None]], axis=-1)     # [G, S, ne + 1]
+                p = entmax_bisect(gamma * z, alpha)                     # [G, S, ne (+1)]
                 tau = entmax_threshold(gamma * z, alpha)                # [G, S]
-                margin = np.abs((alpha - 1.0) * gamma * z - tau[..., None])
-                w[bi, g, sel, :ne] = p.mean(axis=0)
-                near[bi, g, sel, :ne] = (margin < near_tol).any(axis=0)
+                nr = (np.abs((alpha - 1.0) * gamma * z - tau[..., None]) < near_tol).any(axis=0)
+                w[bi, g, sel, :ne] = p[..., :ne].mean(axis=0)
+                near[bi, g, sel, :ne] = nr[..., :ne]
+                if with_diag:
+                    w[bi, g, sel, c_i] = p[..., ne].mean(axis=0)
+                    near[bi, g, sel, c_i] = nr[..., ne]
                 if return_heads:
-                    heads[bi, g * G:(g + 1) * G][:, sel, :ne] = p
-    mask = pack_mask(w > 0.0)
+                    hsl = heads[bi, g * G:(g + 1) * G]
+                    hsl[:, sel, :ne] = p[..., :ne]
+                    if with_diag:
+                        hsl[:, sel, c_i] = p[..., ne]
+    routed = w > 0.0
+    if diag is not None:
+        for k, c_i in enumerate(chunk_of):
+            if c_i < n_c:
+                routed[:, :, k, c_i] = False
+    mask = pack_mask(routed)
     if return_heads:
         return w, mask, near, heads
     return w, mask, near
@@ -353,13 +415,17 @@ def attn_fwd(Q, K, V, w, mask, sigma, B, positions=None):
 # Decode: one new query per sequence against a cached KV and summary cache
 # ----------------------------------------------------------------------------
 
-def decode(q, Kc, Vc, Kbar, L, alpha, gamma, sigma, B, near_tol=1e-4):
+def decode(q, Kc, Vc, Kbar, L, alpha, gamma, sigma, B, near_tol=1e-4, qbar=None):
     """Single-query step at position L-1 of an L-token cache.
 
     q: [b, H_q, d]; Kc, Vc: [b, H_kv, >= L, d]; Kbar: [b, H_kv, >= (L-1)//B, d]
     (summaries of complete chunks; only chunks before the query's own are
     read).  Returns (o [b, H_q, d], lse [b, H_q], w [b, H_kv, n_c],
     mask [b, H_kv, n_w], near [b, H_kv, n_c]) with n_c = ceil(L / B).
+    With qbar [H_kv, d] given, estimate_diagonal is on, as in ``route``: the
+    query's own chunk c_q joins the entmax with the logit of
+    ``diagonal_summary`` over the cache rows c_q B .. L - 1, its weight goes
+    to w[..., c_q] and its mask bit stays clear.
     """
     q, Kc, Vc, Kbar = _f64(q), _f64(Kc), _f64(Vc), _f64(Kbar)
     b, hq, d = q.shape
@@ -375,19 +441,27 @@ def decode(q, Kc, Vc, Kbar, L, alpha, gamma, sigma, B, near_tol=1e-4):
     for bi in range(b):
         for g in range(hkv):
             qg = q[bi, g * G:(g + 1) * G]
-            if c_q > 0:
-                z = qg @ Kbar[bi, g, :c_q].T                        # [G, c_q]
+            z = qg @ Kbar[bi, g, :c_q].T                            # [G, c_q]
+            if qbar is not None:
+                est = diagonal_summary(Kc[bi, g:g + 1, :L], _f64(qbar)[g:g + 1], B, i)[0]
+                z = np.concatenate([z, (qg @ est)[:, None]], axis=1)  # [G, c_q + 1]
+            if z.shape[1] > 0:
                 p = entmax_bisect(gamma * z, alpha)
                 tau = entmax_threshold(gamma * z, alpha)
-                w[bi, g, :c_q] = p.mean(axis=0)
-                near[bi, g, :c_q] = (np.abs((alpha - 1.0) * gamma * z - tau[:, None]) < near_tol).any(axis=0)
-            og, lg = _attend(qg, Kc[bi, g, :L], Vc[bi, g, :L], w[bi, g], w[bi, g] > 0.0, i, B, sigma)
+                w[bi, g, :z.shape[1]] = p.mean(axis=0)
+                near[bi, g, :z.shape[1]] = \
+                    (np.abs((alpha - 1.0) * gamma * z - tau[:, None]) < near_tol).any(axis=0)
+            routed = w[bi, g] > 0.0
+            routed[c_q:] = False
+            og, lg = _attend(qg, Kc[bi, g, :L], Vc[bi, g, :L], w[bi, g], routed, i, B, sigma)
             o[bi, g * G:(g + 1) * G] = og
             lse[bi, g * G:(g + 1) * G] = lg
-    return o, lse, w, pack_mask(w > 0.0), near
+    routed = w > 0.0
+    routed[..., c_q:] = False
+    return o, lse, w, pack_mask(routed), near
 
 
-def decode_varlen(q, Kc, Vc, Kbar, lens, alpha, gamma, sigma, B, near_tol=1e-4):
+def decode_varlen(q, Kc, Vc, Kbar, lens, alpha, gamma, sigma, B, near_tol=1e-4, qbar=None):
     """Decode step for a batch whose sequences hold different numbers of tokens.
 
     Every sequence takes its own incremental-decoding step (gist.science
@@ -412,14 +486,19 @@ def decode_varlen(q, Kc, Vc, Kbar, lens, alpha, gamma, sigma, B, near_tol=1e-4):
             raise ValueError(f"cache length {L} outside [1, {L_max}]")
         c_q = (L - 1) // B
         ob, lb, wb, _, nb = decode(q[bi:bi + 1], Kc[bi:bi + 1, :, :L], Vc[bi:bi + 1, :, :L],
-                                   Kbar[bi:bi + 1, :, :c_q], L, alpha, gamma, sigma, B, near_tol)
+                                   Kbar[bi:bi + 1, :, :c_q], L, alpha, gamma, sigma, B, near_tol,
+                                   qbar)
         o[bi], lse[bi] = ob[0], lb[0]
         w[bi, :, :wb.shape[2]] = wb[0]
         near[bi, :, :nb.shape[2]] = nb[0]
-    return o, lse, w, pack_mask(w > 0.0), near
+    routed = w > 0.0
+    for bi in range(b):
+        routed[bi, :, (int(lens[bi]) - 1) // B:] = False
+    return o, lse, w, pack_mask(routed), near
 
 
-def decode_paged(q, Kpool, Vpool, Kbar, lens, page_table, alpha, gamma, sigma, B, near_tol=1e-4):
+def decode_paged(q, Kpool, Vpool, Kbar, lens, page_table, alpha, gamma, sigma, B, near_tol=1e-4,
+                 qbar=None):
     """``decode_varlen`` on caches kept as pages of one chunk each.
 
     Kpool, Vpool: [n_pages, H_kv, B, d]; page_table[bi, c] is the pool page
@@ -434,7 +513,7 @@ def decode_paged(q, Kpool, Vpool, Kbar, lens, page_table, alpha, gamma, sigma, B
     if Bp != B:
         raise ValueError("a page holds one chunk of B tokens")
     Kc, Vc = gather_pages(Kpool, Vpool, lens, page_table, B)
-    return decode_varlen(q, Kc, Vc, Kbar, lens, alpha, gamma, sigma, B, near_tol)
+    return decode_varlen(q, Kc, Vc, Kbar, lens, alpha, gamma, sigma, B, near_tol, qbar)
 
 
 def gather_pages(Kpool, Vpool, lens, page_table, B):

@@ -256,6 +256,101 @@ def test_route_gqa_mean_and_shared_support():
 
 
 # ----------------------------------------------------------------------------
+# estimate_diagonal: the query's own chunk as one more entmax candidate
+# ----------------------------------------------------------------------------
+
+def _diag_case(seed, b=1, hq=4, hkv=2, n=96, d=8, B=16):
+    rng = np.random.default_rng(seed)
+    Q = rng.normal(size=(b, hq, n, d))
+    K = rng.normal(size=(b, hkv, n, d))
+    qbar = rng.normal(size=(hkv, d)) * 0.5
+    return Q, K, qbar, oracle.chunk_summary(K, qbar, B)
+
+
+def test_route_diag_weights_mask_and_first_chunk():
+    B = 16
+    Q, K, qbar, Kbar = _diag_case(40, b=2)
+    n = Q.shape[2]
+    w, mask, _, heads = oracle.route(Q, Kbar, 1.5, 1.0, B, diag=(K, qbar), return_heads=True)
+    c_i = np.arange(n) // B
+    act = oracle.unpack_mask(mask, Kbar.shape[2])
+    for i in range(n):
+        # the routed chunks and the diagonal share the unit mass
+        np.testing.assert_allclose(w[:, :, i, :c_i[i] + 1].sum(-1), 1.0, atol=1e-12)
+        assert not w[:, :, i, c_i[i] + 1:].any()
+        # the mask holds the routed chunks only, never the query's own chunk
+        assert np.array_equal(act[:, :, i, :c_i[i]], w[:, :, i, :c_i[i]] > 0)
+        assert not act[:, :, i, c_i[i]:].any()
+    # rows of the first chunk: the diagonal is the only candidate
+    np.testing.assert_allclose(w[:, :, :B, 0], 1.0, atol=1e-12)
+    np.testing.assert_allclose(heads[:, :, :B, 0], 1.0, atol=1e-12)
+    # w is the group mean of the per-head weights, diagonal column included
+    np.testing.assert_allclose(w, heads.reshape(2, 2, 2, n, -1).mean(axis=2), atol=1e-15)
+
+
+def test_route_diag_hand_computed_sparsemax():
+    # alpha = 2 (sparsemax), one head, B = 2: for two candidates x0, x1 with
+    # |x0 - x1| < 1 the weights are ((x0 - x1 + 1) / 2, (x1 - x0 + 1) / 2)
+    rng = np.random.default_rng(41)
+    B, d, gamma = 2, 4, 0.3
+    Q = rng.normal(size=(1, 1, 4, d))
+    K = rng.normal(size=(1, 1, 4, d))
+    qbar = rng.normal(size=(1, d))
+    Kbar = oracle.chunk_summary(K, qbar, B)
+    w, mask, _ = oracle.route(Q, Kbar, 2.0, gamma, B, diag=(K, qbar))
+    for i in (2, 3):
+        # position 2 sees key 2 alone (estimate = k2); position 3 sees keys 2, 3
+        s = np.array([qbar[0] @ K[0, 0, 2], qbar[0] @ K[0, 0, 3]]) / math.sqrt(d)
+        a = np.exp(s[: i - 1] - s[: i - 1].max())
+        est = (a / a.sum()) @ K[0, 0, 2:i + 1]
+        x0 = gamma * (Q[0, 0, i] @ Kbar[0, 0, 0])
+        x1 = gamma * (Q[0, 0, i] @ est)
+        if abs(x0 - x1) < 1.0:
+            want = [(x0 - x1 + 1) / 2, (x1 - x0 + 1) / 2]
+        else:
+            want = [1.0, 0.0] if x0 > x1 else [0.0, 1.0]
+        np.testing.assert_allclose(w[0, 0, i, :2], want, atol=1e-12)
+        assert oracle.unpack_mask(mask[0, 0, i], 2)[0] == (want[0] > 0)
+    np.testing.assert_allclose(w[0, 0, :2, 0], 1.0, atol=1e-12)
+
+
+def test_route_diag_at_a_chunk_end_is_plain_routing_a_chunk_later():
+    # at the last row of chunk c the estimate covers the whole chunk, i.e. it
+    # is the summary K_bar_c; routing there equals plain routing (no diagonal
+    # candidate) of the same query one position later, where chunk c has
+    # become an eligible chunk
+    B = 16
+    Q, K, qbar, Kbar = _diag_case(42, n=96)
+    for c in (0, 2, 4):
+        i = (c + 1) * B - 1
+        Q2 = Q.copy()
+        Q2[:, :, i + 1] = Q[:, :, i]
+        wd, _, _ = oracle.route(Q, Kbar, 1.5, 1.0, B, positions=[i], diag=(K, qbar))
+        wp, _, _ = oracle.route(Q2, Kbar, 1.5, 1.0, B, positions=[i + 1])
+        np.testing.assert_allclose(wd[:, :, 0, :c + 1], wp[:, :, 0, :c + 1], atol=1e-12)
+
+
+def test_decode_diag_is_the_last_routed_row():
+    B, L = 16, 90
+    Q, K, qbar, Kbar = _diag_case(43, b=2, n=96)
+    rng = np.random.default_rng(44)
+    V = rng.normal(size=K.shape)
+    w, mask, _ = oracle.route(Q, Kbar, 1.5, 0.9, B, positions=[L - 1], diag=(K, qbar))
+    O, lse = oracle.attn_fwd(Q, K, V, w, mask, 0.7, B, positions=[L - 1])
+    o, lse_d, wd, md, _ = oracle.decode(Q[:, :, L - 1], K, V, Kbar, L, 1.5, 0.9, 0.7, B, qbar=qbar)
+    n_c = wd.shape[-1]
+    np.testing.assert_allclose(wd, w[:, :, 0, :n_c], atol=1e-12)
+    assert np.array_equal(oracle.unpack_mask(md, n_c), oracle.unpack_mask(mask[:, :, 0], 6)[..., :n_c])
+    np.testing.assert_allclose(o, O[:, :, 0], atol=1e-12)
+    np.testing.assert_allclose(lse_d, lse[:, :, 0], atol=1e-12)
+    # a length per sequence reduces to the fixed-length call, pages to contiguous
+    got = oracle.decode_varlen(Q[:, :, L - 1], K[:, :, :L], V[:, :, :L], Kbar, [L, L], 1.5, 0.9,
+                               0.7, B, qbar=qbar)
+    for a, b_ in zip(got, (o, lse_d, wd, md)):
+        np.testing.assert_array_equal(a, b_)
+
+
+# ----------------------------------------------------------------------------
 # Stage 2
 # ----------------------------------------------------------------------------
 
