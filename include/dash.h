@@ -71,6 +71,7 @@ typedef struct {
   float gamma;          /* routing logit scale, finite and > 0 */
   float sigma;          /* prior strength, finite and >= 0 */
   int32_t dtype;        /* dash_dtype */
+  int32_t estimate_diagonal;  /* 0 or 1; see dash_route */
 } dash_problem;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -124,9 +125,23 @@ int dash_summarize_append(const dash_problem* p, const int32_t* cache_lens,
  *   w[b, g, i, c] = mean of p over the G query heads of KV head g
  *   mask bit      = (w > 0), i.e. the union of the member supports.
  * Entries for c >= c_i are written as 0.  Requires n_c <= 2048.
+ *
+ * p->estimate_diagonal = 1 (aiexpert.news, interface paragraph: a flag for a
+ * diagonal correction of the alpha-entmax normalisation; gist.science
+ * summary, Fase 2 "Diagonaal Afhandeling": the chunk on the diagonal has no
+ * summary yet): the query's own chunk c_i joins the entmax as one more
+ * candidate, z[h, c_i] = Q[b, h, i] . Khat_i, where Khat_i is stage 0's
+ * learned-query summary of the keys K[b, g, c_i B .. i] (the part of the
+ * chunk the query sees), computed here in fp32 and not stored.  Its group
+ * mean goes to w[b, g, i, c_i] (so the routed chunks share 1 - w[.., c_i]);
+ * mask bit c_i stays clear: stage 2 attends to the query's own chunk with
+ * weight 1 whatever w[.., c_i] is.  Rows of the first chunk get
+ * w[.., 0] = 1.  K [b, Hkv, N, d] (dtype of Q) and qbar [Hkv, d] fp32 are
+ * then required (16-byte aligned); with estimate_diagonal = 0 they are
+ * ignored and may be NULL.
  */
-int dash_route(const dash_problem* p, const void* Q, const void* Kbar,
-               float* w, uint32_t* mask, void* stream);
+int dash_route(const dash_problem* p, const void* Q, const void* Kbar, const void* K,
+               const float* qbar, float* w, uint32_t* mask, void* stream);
 
 /*
  * Fixed-budget top-k routing on the same summaries: the baseline the pages
@@ -141,8 +156,9 @@ int dash_route(const dash_problem* p, const void* Q, const void* Kbar,
  * softmax attention on the selected chunks plus the diagonal chunk, with the
  * same stage-2 kernel.  A reference kernel on CUDA cores (one warp per row),
  * not a tuned router.
- * Errors: as dash_route; k < 1 -> DASH_ERR_INVALID_ARG; G > 16 or more than
- * 2048 chunks -> DASH_ERR_UNSUPPORTED.
+ * Errors: as dash_route; k < 1 -> DASH_ERR_INVALID_ARG; G > 16, more than
+ * 2048 chunks or p->estimate_diagonal = 1 (there is no entmax normalisation
+ * to correct) -> DASH_ERR_UNSUPPORTED.
  */
 int dash_route_topk(const dash_problem* p, const void* Q, const void* Kbar, int k, float* w,
                     uint32_t* mask, void* stream);
@@ -200,7 +216,9 @@ int dash_attn_bwd(const dash_problem* p, const void* Q, const void* K, const voi
  *   ACCUMULATED into (dQ after dash_attn_bwd wrote it; dKbar zeroed by the
  *   caller; dKbar by atomics).
  * Reference kernel on CUDA cores (one warp per position and KV head, the
- * threshold recomputed by bisection).  Errors: as dash_route.
+ * threshold recomputed by bisection).  Errors: as dash_route;
+ * p->estimate_diagonal = 1 -> DASH_ERR_UNSUPPORTED (the gradient through the
+ * diagonal candidate is not built).
  */
 int dash_route_bwd(const dash_problem* p, const void* Q, const void* Kbar, const float* dw,
                    float* dQ, float* dKbar, void* stream);
@@ -230,12 +248,16 @@ size_t dash_workspace_bytes(const dash_problem* p, int is_decode);
  *   o [b, Hq, d]; lse [b, Hq] (nullable); w [b, Hkv, n_c] (nullable);
  *   mask [b, Hkv, n_w] (nullable).
  * Equals row L - 1 of stage 1 + stage 2 on the same data.
+ * qbar [Hkv, d] fp32: required with p->estimate_diagonal = 1 (the query's
+ * own chunk c_q joins the entmax with stage 0's summary of the cache rows
+ * c_q B .. L - 1, as in dash_route; its weight goes to w[.., c_q] and is not
+ * a mask bit), else ignored and may be NULL.
  * workspace: dash_workspace_bytes(p, 1) bytes, 256-byte aligned.
  */
 int dash_decode(const dash_problem* p, const void* q, const void* Kcache,
-                const void* Vcache, const void* Kbar, void* o, float* lse,
-                float* w, uint32_t* mask, void* workspace, size_t workspace_bytes,
-                void* stream);
+                const void* Vcache, const void* Kbar, const float* qbar, void* o,
+                float* lse, float* w, uint32_t* mask, void* workspace,
+                size_t workspace_bytes, void* stream);
 
 /*
  * Decode for a batch of sequences with different cache lengths (each at its
@@ -257,9 +279,9 @@ int dash_decode(const dash_problem* p, const void* q, const void* Kcache,
  * dash_get_error return DASH_ERR_INVALID_ARG.
  */
 int dash_decode_varlen(const dash_problem* p, const int32_t* cache_lens, const void* q,
-                       const void* Kcache, const void* Vcache, const void* Kbar, void* o,
-                       float* lse, float* w, uint32_t* mask, void* workspace,
-                       size_t workspace_bytes, void* stream);
+                       const void* Kcache, const void* Vcache, const void* Kbar,
+                       const float* qbar, void* o, float* lse, float* w, uint32_t* mask,
+                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * dash_decode_varlen over paged K/V caches, the layout a serving engine keeps
@@ -269,8 +291,9 @@ int dash_decode_varlen(const dash_problem* p, const int32_t* cache_lens, const v
  *   [b, max_pages], 4-byte aligned, max_pages >= ceil(L_max / B): chunk c of
  *   sequence bi is pool page page_table[bi * max_pages + c] (entries for
  *   chunks at or past ceil(L_b / B) are never read; pages may be shared).
- *   cache_lens, Kbar (still one contiguous summary cache per sequence), q, o,
- *   lse, w, mask, workspace: as in dash_decode_varlen with L_max = p->seq_len.
+ *   cache_lens, Kbar (still one contiguous summary cache per sequence), qbar,
+ *   q, o, lse, w, mask, workspace: as in dash_decode_varlen with
+ *   L_max = p->seq_len.
  * Equals dash_decode_varlen on the caches the pages spell out.
  * Errors: those of dash_decode_varlen; page_table NULL or misaligned,
  * max_pages < ceil(L_max / B) or n_pages < 1 -> DASH_ERR_INVALID_ARG;
@@ -281,8 +304,9 @@ int dash_decode_varlen(const dash_problem* p, const int32_t* cache_lens, const v
  */
 int dash_decode_paged(const dash_problem* p, const int32_t* cache_lens, const int32_t* page_table,
                       int max_pages, int n_pages, const void* q, const void* Kpool,
-                      const void* Vpool, const void* Kbar, void* o, float* lse, float* w,
-                      uint32_t* mask, void* workspace, size_t workspace_bytes, void* stream);
+                      const void* Vpool, const void* Kbar, const float* qbar, void* o,
+                      float* lse, float* w, uint32_t* mask, void* workspace,
+                      size_t workspace_bytes, void* stream);
 
 /*
  * Decode without a caller-provided workspace.  The pages on DashAttention
@@ -291,7 +315,8 @@ int dash_decode_paged(const dash_problem* p, const int32_t* cache_lens, const in
  * GPU to its own pool, or a plugin interface that forbids allocation, cannot
  * supply the dash_workspace_bytes(p, 1) scratch that dash_decode needs.
  *
- * Same arguments, result and errors as dash_decode, minus the workspace.
+ * Same arguments, result and errors as dash_decode, minus the workspace and
+ * qbar (p->estimate_diagonal = 1 returns DASH_ERR_UNSUPPORTED).
  * The scratch is a fixed 8 MiB array in device memory, reserved on every GPU
  * that loads this library until the process exits; no cudaMalloc/cudaFree or
  * other allocating routine is called.  Every problem dash_decode accepts

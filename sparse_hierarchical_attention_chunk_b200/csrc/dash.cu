@@ -41,6 +41,7 @@ int check_problem(const dash_problem* p, bool decode) {
   if (!(p->gamma > 0.f) || !isfinite(p->gamma)) return DASH_ERR_INVALID_ARG;
   if (!(p->sigma >= 0.f) || !isfinite(p->sigma)) return DASH_ERR_INVALID_ARG;
   if (p->dtype != DASH_F32 && p->dtype != DASH_BF16) return DASH_ERR_INVALID_ARG;
+  if (p->estimate_diagonal != 0 && p->estimate_diagonal != 1) return DASH_ERR_INVALID_ARG;
   // sizes must fit the 32-bit row indices used by the kernels and TMA
   const long long rows = (long long)p->batch * p->n_q_heads * p->seq_len;
   if (rows > (1ll << 31) - 1) return DASH_ERR_UNSUPPORTED;
@@ -119,7 +120,7 @@ const char* dash_status_str(int s) {
   }
 }
 
-int dash_version(void) { return (1 << 16) | 0; }
+int dash_version(void) { return (2 << 16) | 0; }
 
 int dash_summarize(const dash_problem* p, const void* K, const float* qbar, int chunk_begin,
                    int chunk_end, void* Kbar, void* stream) {
@@ -180,6 +181,7 @@ int dash_route_topk(const dash_problem* p, const void* Q, const void* Kbar, int 
       !aligned16(mask) || k < 1)
     return DASH_ERR_INVALID_ARG;
   if (n_chunks(p) > dash::kTopkMaxChunks || p->n_q_heads / p->n_kv_heads > 16) return DASH_ERR_UNSUPPORTED;
+  if (p->estimate_diagonal) return DASH_ERR_UNSUPPORTED;   // no entmax normalisation to correct
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
 #define DASH_TOPK(T, D)                                                                         \
@@ -230,6 +232,7 @@ int dash_route_bwd(const dash_problem* p, const void* Q, const void* Kbar, const
   for (const void* ptr : req)
     if (!ptr || !aligned16(ptr)) return DASH_ERR_INVALID_ARG;
   if (p->n_q_heads / p->n_kv_heads > 16 || n_chunks(p) > dash::kRbMaxChunks) return DASH_ERR_UNSUPPORTED;
+  if (p->estimate_diagonal) return DASH_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
 #define DASH_RB(T, D)                                                                            \
@@ -264,25 +267,31 @@ int dash_summarize_bwd(const dash_problem* p, const void* K, const float* qbar, 
   return cuda_status(e);
 }
 
-int dash_route(const dash_problem* p, const void* Q, const void* Kbar, float* w, uint32_t* mask,
-               void* stream) {
+int dash_route(const dash_problem* p, const void* Q, const void* Kbar, const void* K,
+               const float* qbar, float* w, uint32_t* mask, void* stream) {
   int rc = check_problem(p, false);
   if (rc) return rc;
   if (!Q || !Kbar || !w || !mask || !aligned16(Q) || !aligned16(Kbar) || !aligned16(w) ||
       !aligned16(mask))
     return DASH_ERR_INVALID_ARG;
+  if (p->estimate_diagonal && (!K || !qbar || !aligned16(K) || !aligned16(qbar)))
+    return DASH_ERR_INVALID_ARG;
   if (n_chunks(p) > 2048) return DASH_ERR_UNSUPPORTED;
+  if (!p->estimate_diagonal) {
+    K = nullptr;
+    qbar = nullptr;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
 #define DASH_ROUTE(T, D)                                                                      \
   dash::launch_route<T, D>(static_cast<const T*>(Q), static_cast<const T*>(Kbar), w, mask,    \
-                           p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, p->chunk,       \
-                           p->alpha, p->gamma, st)
+                           static_cast<const T*>(K), qbar, p->batch, p->n_q_heads,            \
+                           p->n_kv_heads, p->seq_len, p->chunk, p->alpha, p->gamma, st)
   const int G = p->n_q_heads / p->n_kv_heads;
   if (p->dtype == DASH_BF16 && p->head_dim == 128 && G == 16 && n_chunks(p) <= 1024)
     e = dash::launch_route_tc(static_cast<const bf16*>(Q), static_cast<const bf16*>(Kbar), w, mask,
-                              p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, p->chunk,
-                              p->alpha, p->gamma, st);
+                              static_cast<const bf16*>(K), qbar, p->batch, p->n_q_heads,
+                              p->n_kv_heads, p->seq_len, p->chunk, p->alpha, p->gamma, st);
   else if (p->dtype == DASH_BF16)
     e = p->head_dim == 128 ? DASH_ROUTE(bf16, 128) : DASH_ROUTE(bf16, 64);
   else
@@ -337,12 +346,14 @@ int dash_attn_fwd(const dash_problem* p, const void* Q, const void* K, const voi
 // dash_decode_paged (page_table: nullable device [batch][max_pages])
 static int decode_entry(const dash_problem* p, const int32_t* lens, const int32_t* page_table,
                         int max_pages, int n_pages, const void* q,
-                        const void* Kcache, const void* Vcache, const void* Kbar, void* o,
-                        float* lse, float* w, uint32_t* mask, void* workspace,
-                        size_t workspace_bytes, void* stream) {
+                        const void* Kcache, const void* Vcache, const void* Kbar,
+                        const float* qbar, void* o, float* lse, float* w, uint32_t* mask,
+                        void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_problem(p, true);
   if (rc) return rc;
   if (!q || !Kcache || !Vcache || !Kbar || !o) return DASH_ERR_INVALID_ARG;
+  if (p->estimate_diagonal && (!qbar || !aligned16(qbar))) return DASH_ERR_INVALID_ARG;
+  if (!p->estimate_diagonal) qbar = nullptr;
   if (!aligned16(q) || !aligned16(Kcache) || !aligned16(Vcache) || !aligned16(Kbar) ||
       !aligned16(o) || (lse && !aligned16(lse)) || (w && !aligned16(w)) || (mask && !aligned16(mask)))
     return DASH_ERR_INVALID_ARG;
@@ -357,32 +368,33 @@ static int decode_entry(const dash_problem* p, const int32_t* lens, const int32_
                         p->chunk, p->alpha, p->gamma, p->sigma, lens, page_table, max_pages,
                         n_pages, static_cast<const bf16*>(q),
                         static_cast<const bf16*>(Kcache), static_cast<const bf16*>(Vcache),
-                        static_cast<const bf16*>(Kbar), static_cast<bf16*>(o), lse, w, mask,
-                        workspace, static_cast<cudaStream_t>(stream));
+                        static_cast<const bf16*>(Kbar), qbar, static_cast<bf16*>(o), lse, w,
+                        mask, workspace, static_cast<cudaStream_t>(stream));
   if (rc == DASH_ERR_CUDA) (void)cudaGetLastError();
   return rc;
 }
 
 int dash_decode(const dash_problem* p, const void* q, const void* Kcache, const void* Vcache,
-                const void* Kbar, void* o, float* lse, float* w, uint32_t* mask, void* workspace,
-                size_t workspace_bytes, void* stream) {
-  return decode_entry(p, nullptr, nullptr, 0, 0, q, Kcache, Vcache, Kbar, o, lse, w, mask,
+                const void* Kbar, const float* qbar, void* o, float* lse, float* w,
+                uint32_t* mask, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_entry(p, nullptr, nullptr, 0, 0, q, Kcache, Vcache, Kbar, qbar, o, lse, w, mask,
                       workspace, workspace_bytes, stream);
 }
 
 int dash_decode_varlen(const dash_problem* p, const int32_t* cache_lens, const void* q,
-                       const void* Kcache, const void* Vcache, const void* Kbar, void* o,
-                       float* lse, float* w, uint32_t* mask, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+                       const void* Kcache, const void* Vcache, const void* Kbar,
+                       const float* qbar, void* o, float* lse, float* w, uint32_t* mask,
+                       void* workspace, size_t workspace_bytes, void* stream) {
   if (!cache_lens || (reinterpret_cast<uintptr_t>(cache_lens) & 3u)) return DASH_ERR_INVALID_ARG;
-  return decode_entry(p, cache_lens, nullptr, 0, 0, q, Kcache, Vcache, Kbar, o, lse, w, mask,
-                      workspace, workspace_bytes, stream);
+  return decode_entry(p, cache_lens, nullptr, 0, 0, q, Kcache, Vcache, Kbar, qbar, o, lse, w,
+                      mask, workspace, workspace_bytes, stream);
 }
 
 int dash_decode_paged(const dash_problem* p, const int32_t* cache_lens, const int32_t* page_table,
                       int max_pages, int n_pages, const void* q, const void* Kpool,
-                      const void* Vpool, const void* Kbar, void* o, float* lse, float* w,
-                      uint32_t* mask, void* workspace, size_t workspace_bytes, void* stream) {
+                      const void* Vpool, const void* Kbar, const float* qbar, void* o, float* lse,
+                      float* w, uint32_t* mask, void* workspace, size_t workspace_bytes,
+                      void* stream) {
   int rc = check_problem(p, true);
   if (rc) return rc;
   if (!cache_lens || (reinterpret_cast<uintptr_t>(cache_lens) & 3u) || !page_table ||
@@ -391,8 +403,8 @@ int dash_decode_paged(const dash_problem* p, const int32_t* cache_lens, const in
   if (max_pages < n_chunks(p) || n_pages < 1) return DASH_ERR_INVALID_ARG;
   // TMA row coordinates are 32-bit
   if ((long long)n_pages * p->n_kv_heads * p->chunk > 0x7fffffffLL) return DASH_ERR_UNSUPPORTED;
-  return decode_entry(p, cache_lens, page_table, max_pages, n_pages, q, Kpool, Vpool, Kbar, o,
-                      lse, w, mask, workspace, workspace_bytes, stream);
+  return decode_entry(p, cache_lens, page_table, max_pages, n_pages, q, Kpool, Vpool, Kbar, qbar,
+                      o, lse, w, mask, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"
@@ -468,7 +480,7 @@ int dash_decode_noalloc(const dash_problem* p, const void* q, const void* Kcache
   if (!aligned16(q) || !aligned16(Kcache) || !aligned16(Vcache) || !aligned16(Kbar) ||
       !aligned16(o) || (lse && !aligned16(lse)) || (w && !aligned16(w)) || (mask && !aligned16(mask)))
     return DASH_ERR_INVALID_ARG;
-  if (p->dtype != DASH_BF16) return DASH_ERR_UNSUPPORTED;
+  if (p->dtype != DASH_BF16 || p->estimate_diagonal) return DASH_ERR_UNSUPPORTED;
   const int G = p->n_q_heads / p->n_kv_heads;
   if (G > 16 || n_chunks(p) > 2048 || p->batch * p->n_kv_heads > 64) return DASH_ERR_UNSUPPORTED;
   const size_t need = dash::decode_workspace_bytes(p->batch, p->n_q_heads, p->n_kv_heads,
@@ -483,8 +495,8 @@ int dash_decode_noalloc(const dash_problem* p, const void* q, const void* Kcache
                         p->chunk, p->alpha, p->gamma, p->sigma, nullptr, nullptr, 0, 0,
                         static_cast<const bf16*>(q),
                         static_cast<const bf16*>(Kcache), static_cast<const bf16*>(Vcache),
-                        static_cast<const bf16*>(Kbar), static_cast<bf16*>(o), lse, w, mask,
-                        scratch, static_cast<cudaStream_t>(stream));
+                        static_cast<const bf16*>(Kbar), nullptr, static_cast<bf16*>(o), lse, w,
+                        mask, scratch, static_cast<cudaStream_t>(stream));
   if (rc == DASH_ERR_CUDA) (void)cudaGetLastError();
   return rc;
 }

@@ -231,6 +231,12 @@ struct DecodeRouteParams {
   float* blist;
   int* counts;
   const int* lens;             // nullable: cache length per sequence (else L for all)
+  // estimate_diagonal (diag != 0): the key cache (or page pool with
+  // page_table) and the learned queries of stage 0
+  const __nv_bfloat16* Kc;
+  const float* qbar;
+  const int* page_table;
+  int max_pages, n_pages, diag;
   int n_q, n_kv, kbar_rows, n_c, L, chunk;
   float xscale, e, sigma;
 };
@@ -252,6 +258,7 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
   __shared__ __align__(16) float red[2][2][4][4];   // float4 rows (Group4::sum4)
   __shared__ int cnt_all[kRouteCluster];
   __shared__ int wcnt[8];
+  __shared__ float khat[D];                   // estimate_diagonal: the query chunk's summary
 
   const int r = (int)cluster.block_rank();
   const int bg = blockIdx.x / kRouteCluster;
@@ -338,9 +345,40 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
       }
     }
   }
+  // ---- estimate_diagonal: the query's own chunk c_q as one more candidate,
+  // its logit against stage 0's summary of the cache rows c_q B .. L_b - 1,
+  // stored by the CTA that owns each head in X[slot][c_q]
+  const bool dg = prm.diag != 0 && c_q > 0;
+  if (dg && r * HPC < G) {                      // uniform over the CTA
+    if (warp == 0) {
+      const __nv_bfloat16* rows;
+      if (prm.page_table) {
+        int pg = __ldg(prm.page_table + (size_t)b * prm.max_pages + c_q);
+        if (pg < 0 || pg >= prm.n_pages) {
+          if (lane == 0) atomicOr(&g_dash_error, DASH_DEV_ERR_ARG);
+          pg = 0;
+        }
+        rows = prm.Kc + ((size_t)pg * prm.n_kv + g) * prm.chunk * D;
+      } else {
+        rows = prm.Kc + ((size_t)bg * prm.L + (size_t)c_q * prm.chunk) * D;
+      }
+      summarize_chunk_warp<__nv_bfloat16, D, 4, float>(rows, prm.qbar + g * D, khat,
+                                                      Lb - c_q * prm.chunk, lane);
+    }
+    __syncthreads();
+    const int h = r * HPC + warp;
+    if (warp < HPC && h < G) {
+      const __nv_bfloat16* qh = prm.q + ((size_t)b * prm.n_q + g * G + h) * D;
+      float acc = 0.f;
+      for (int j = lane; j < D; j += 32) acc = fmaf(__bfloat162float(qh[j]), khat[j], acc);
+      acc = warp_sum(acc);
+      if (lane == 0) X[warp][c_q] = acc * prm.xscale;
+    }
+  }
   cluster.sync();
 
   // ---- entmax of the owned heads, four warps per head -> p to the chunk owners
+  const int n_cand = c_q + (dg ? 1 : 0);        // candidates: eligible chunks (+ the diagonal)
   {
     const int slot = warp >> 2;
     const int h = r * HPC + slot;
@@ -350,14 +388,14 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
 #pragma unroll
       for (int k = 0; k < NV; ++k) {
         const int c = tg + 128 * k;
-        x[k] = c < c_q ? X[slot][c] : -INFINITY;
+        x[k] = c < n_cand ? X[slot][c] : -INFINITY;
       }
       Group4 gr{red[slot], warp & 3, lane, 1 + slot, 0};
       const float tau = entmax_tau_group<NV, KIND>(x, prm.e, gr);
 #pragma unroll
       for (int k = 0; k < NV; ++k) {
         const int c = tg + 128 * k;
-        if (c < c_q) {
+        if (c < n_cand) {
           const float pv = entmax_pow<KIND>(fmaxf(x[k] - tau, 0.f), prm.e);
           const int owner = c / CPC;
           float* dst = cluster.map_shared_rank(&Pp[h][c - owner * CPC], owner);
@@ -373,13 +411,15 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
   float wv = 0.f;
   bool act = false;
   if (tid < CPC && c < prm.n_c) {
-    if (c < c_q) {
+    if (c < n_cand) {
       float s = 0.f;
       for (int hh = 0; hh < G; ++hh) s += Pp[hh][tid];
       wv = s / (float)G;
+    } else if (prm.diag && c == c_q && c_q == 0) {
+      wv = 1.f;                                   // the diagonal is the only candidate
     }
     if (prm.w) prm.w[(size_t)bg * prm.n_c + c] = wv;
-    act = wv > 0.f;
+    act = wv > 0.f && c < c_q;                    // the query's own chunk is never routed
   }
   const unsigned bal = __ballot_sync(0xffffffffu, act);
   const int nw = (prm.n_c + 31) >> 5;
@@ -975,11 +1015,14 @@ inline int decode_split_ctas(int n_bg, int c_q, int sms) {
 // L is then the caches' capacity.  page_table: nullable device array
 // [batch][max_pages]; with it Kc and Vc are page pools [n_pages][n_kv][chunk][D]
 // and chunk c of sequence b is pool page page_table[b][c].
+// qbar: nullable; non-null turns on estimate_diagonal (the learned queries of
+// stage 0, [n_kv][D] fp32).
 inline int run_decode(int batch, int n_q, int n_kv, int L, int D, int chunk, float alpha,
                       float gamma, float sigma, const int* lens, const int* page_table,
                       int max_pages, int n_pages, const __nv_bfloat16* q, const __nv_bfloat16* Kc,
-                      const __nv_bfloat16* Vc, const __nv_bfloat16* Kbar, __nv_bfloat16* o,
-                      float* lse, float* w, uint32_t* mask, void* workspace, cudaStream_t st) {
+                      const __nv_bfloat16* Vc, const __nv_bfloat16* Kbar, const float* qbar,
+                      __nv_bfloat16* o, float* lse, float* w, uint32_t* mask, void* workspace,
+                      cudaStream_t st) {
   const int n_bg = batch * n_kv;
   const int n_c = (L + chunk - 1) / chunk;
   if (n_bg > 64 || n_c > kDecodeMaxChunks || n_q / n_kv > 16) return 2;   // DASH_ERR_UNSUPPORTED
@@ -1002,6 +1045,12 @@ inline int run_decode(int batch, int n_q, int n_kv, int L, int D, int chunk, flo
   rp.n_q = n_q;
   rp.n_kv = n_kv;
   rp.lens = lens;
+  rp.Kc = Kc;
+  rp.qbar = qbar;
+  rp.page_table = page_table;
+  rp.max_pages = max_pages;
+  rp.n_pages = n_pages;
+  rp.diag = qbar != nullptr;
   rp.kbar_rows = L / chunk;
   rp.n_c = n_c;
   rp.L = L;

@@ -23,6 +23,7 @@
 #pragma once
 
 #include "dash_common.cuh"
+#include "summarize.cuh"
 
 namespace dash {
 
@@ -202,12 +203,18 @@ struct RouteLogits<float, D> {
   }
 };
 
+// estimate_diagonal (K, qbar non-null): the query's own chunk c_i joins each
+// head's entmax as one more candidate; its logit is q . (stage 0's summary of
+// the keys c_i B .. i), its group-mean weight goes to w[c_i] and it never
+// sets a mask bit.
 template <typename T, int D, int NV, int KIND>
 __global__ void __launch_bounds__(256) route_kernel(
     const T* __restrict__ Q, const T* __restrict__ Kbar, float* __restrict__ w,
-    uint32_t* __restrict__ mask, int n_q, int n_kv, int seq, int chunk, int n_c, int kbar_rows,
-    float xscale, float e, int n_bg) {
+    uint32_t* __restrict__ mask, const T* __restrict__ K, const float* __restrict__ qbar,
+    int n_q, int n_kv, int seq, int chunk, int n_c, int kbar_rows, float xscale, float e,
+    int n_bg) {
   extern __shared__ __align__(16) float Ls[];
+  __shared__ float khat[8][D];                 // estimate_diagonal: summary per position
   const int G = n_q / n_kv;
   const int n_tiles = seq >> 3;
   const int tile = n_tiles - 1 - (int)(blockIdx.x / n_bg);   // heavy (late) tiles first
@@ -224,6 +231,15 @@ __global__ void __launch_bounds__(256) route_kernel(
 #pragma unroll
   for (int k = 0; k < NV; ++k) wacc[k] = 0.f;
 
+  const bool diag = K != nullptr;
+  const bool dg = diag && n_elig > 0;
+  if (dg) {
+    // warp p: the visible keys of position pos0 + p in its own chunk
+    summarize_chunk_warp<T, D, 4, float>(K + ((size_t)bg * seq + (size_t)c_i * chunk) * D,
+                                         qbar + g * D, khat[warp], pos0 + warp - c_i * chunk + 1,
+                                         lane);
+    __syncwarp();
+  }
   if (n_elig > 0) {
     for (int h0 = 0; h0 < G; h0 += 2) {
       const bool row1_valid = h0 + 1 < G;
@@ -235,11 +251,18 @@ __global__ void __launch_bounds__(256) route_kernel(
       for (int hsel = 0; hsel < 2; ++hsel) {
         if (hsel == 1 && !row1_valid) break;
         const float* row = Ls + (hsel * 8 + warp) * LS;
+        float xd = -INFINITY;
+        if (dg) {
+          const T* qr = Q + (hsel ? qrow1 : qrow0) + (size_t)warp * D;
+          float acc = 0.f;
+          for (int j = lane; j < D; j += 32) acc = fmaf(Elem<T>::to_f(qr[j]), khat[warp][j], acc);
+          xd = xscale * warp_sum(acc);
+        }
         float x[NV];
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
           const int c = lane + 32 * k;
-          x[k] = c < n_elig ? xscale * row[c] : -INFINITY;
+          x[k] = c < n_elig ? xscale * row[c] : (c == c_i ? xd : -INFINITY);
         }
         const float tau = entmax_tau_warp<NV, KIND>(x, e);
 #pragma unroll
@@ -254,21 +277,23 @@ __global__ void __launch_bounds__(256) route_kernel(
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
     const int c = lane + 32 * k;
-    if (c < n_c) wr[c] = wacc[k] * invG;
+    // a row of the first chunk with the diagonal candidate: weight 1 on it
+    if (c < n_c) wr[c] = diag && n_elig == 0 ? (c == c_i ? 1.f : 0.f) : wacc[k] * invG;
   }
   const int nw = (n_c + 31) >> 5;
   uint32_t* mr = mask + row * nw;
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
     const int c = lane + 32 * k;
-    const unsigned bits = __ballot_sync(0xffffffffu, c < n_c && wacc[k] > 0.f);
+    const unsigned bits = __ballot_sync(0xffffffffu, c < n_c && c < c_i && wacc[k] > 0.f);
     if (k < nw && lane == (k & 31)) mr[k] = bits;
   }
 }
 
 template <typename T, int D, int NV, int KIND>
-cudaError_t launch_route_nv(const T* Q, const T* Kbar, float* w, uint32_t* mask, int batch, int n_q,
-                            int n_kv, int seq, int chunk, float xscale, float e, cudaStream_t st) {
+cudaError_t launch_route_nv(const T* Q, const T* Kbar, float* w, uint32_t* mask, const T* K,
+                            const float* qbar, int batch, int n_q, int n_kv, int seq, int chunk,
+                            float xscale, float e, cudaStream_t st) {
   const int n_c = (seq + chunk - 1) / chunk;
   const int LS = ((n_c + 7) & ~7) + 4;
   const size_t smem = (size_t)16 * LS * sizeof(float);
@@ -277,37 +302,43 @@ cudaError_t launch_route_nv(const T* Q, const T* Kbar, float* w, uint32_t* mask,
   if (err != cudaSuccess) return err;
   const int n_bg = batch * n_kv;
   const unsigned grid = (unsigned)(n_bg * (seq / 8));
-  kern<<<grid, 256, smem, st>>>(Q, Kbar, w, mask, n_q, n_kv, seq, chunk, n_c, seq / chunk, xscale,
-                                e, n_bg);
+  kern<<<grid, 256, smem, st>>>(Q, Kbar, w, mask, K, qbar, n_q, n_kv, seq, chunk, n_c, seq / chunk,
+                                xscale, e, n_bg);
   return cudaGetLastError();
 }
 
 template <typename T, int D, int KIND>
-cudaError_t launch_route_kind(const T* Q, const T* Kbar, float* w, uint32_t* mask, int batch,
-                              int n_q, int n_kv, int seq, int chunk, float xscale, float e,
-                              cudaStream_t st) {
+cudaError_t launch_route_kind(const T* Q, const T* Kbar, float* w, uint32_t* mask, const T* K,
+                              const float* qbar, int batch, int n_q, int n_kv, int seq, int chunk,
+                              float xscale, float e, cudaStream_t st) {
   const int n_c = (seq + chunk - 1) / chunk;
-  if (n_c <= 128)
-    return launch_route_nv<T, D, 4, KIND>(Q, Kbar, w, mask, batch, n_q, n_kv, seq, chunk, xscale, e, st);
-  if (n_c <= 256)
-    return launch_route_nv<T, D, 8, KIND>(Q, Kbar, w, mask, batch, n_q, n_kv, seq, chunk, xscale, e, st);
-  if (n_c <= 512)
-    return launch_route_nv<T, D, 16, KIND>(Q, Kbar, w, mask, batch, n_q, n_kv, seq, chunk, xscale, e, st);
-  if (n_c <= 1024)
-    return launch_route_nv<T, D, 32, KIND>(Q, Kbar, w, mask, batch, n_q, n_kv, seq, chunk, xscale, e, st);
-  return launch_route_nv<T, D, 64, KIND>(Q, Kbar, w, mask, batch, n_q, n_kv, seq, chunk, xscale, e, st);
+#define DASH_RNV(NV)                                                                              \
+  launch_route_nv<T, D, NV, KIND>(Q, Kbar, w, mask, K, qbar, batch, n_q, n_kv, seq, chunk, xscale, \
+                                  e, st)
+  if (n_c <= 128) return DASH_RNV(4);
+  if (n_c <= 256) return DASH_RNV(8);
+  if (n_c <= 512) return DASH_RNV(16);
+  if (n_c <= 1024) return DASH_RNV(32);
+  return DASH_RNV(64);
+#undef DASH_RNV
 }
 
+// K, qbar: non-null for estimate_diagonal (the keys and learned queries of
+// stage 0), else both null
 template <typename T, int D>
-cudaError_t launch_route(const T* Q, const T* Kbar, float* w, uint32_t* mask, int batch, int n_q,
-                         int n_kv, int seq, int chunk, float alpha, float gamma, cudaStream_t st) {
+cudaError_t launch_route(const T* Q, const T* Kbar, float* w, uint32_t* mask, const T* K,
+                         const float* qbar, int batch, int n_q, int n_kv, int seq, int chunk,
+                         float alpha, float gamma, cudaStream_t st) {
   const float xscale = (alpha - 1.f) * gamma;
   const float e = 1.f / (alpha - 1.f);
   if (alpha == 1.5f)
-    return launch_route_kind<T, D, kEntmax15>(Q, Kbar, w, mask, batch, n_q, n_kv, seq, chunk, xscale, e, st);
+    return launch_route_kind<T, D, kEntmax15>(Q, Kbar, w, mask, K, qbar, batch, n_q, n_kv, seq,
+                                               chunk, xscale, e, st);
   if (alpha == 2.f)
-    return launch_route_kind<T, D, kSparsemax>(Q, Kbar, w, mask, batch, n_q, n_kv, seq, chunk, xscale, e, st);
-  return launch_route_kind<T, D, kEntmaxGeneric>(Q, Kbar, w, mask, batch, n_q, n_kv, seq, chunk, xscale, e, st);
+    return launch_route_kind<T, D, kSparsemax>(Q, Kbar, w, mask, K, qbar, batch, n_q, n_kv, seq,
+                                                chunk, xscale, e, st);
+  return launch_route_kind<T, D, kEntmaxGeneric>(Q, Kbar, w, mask, K, qbar, batch, n_q, n_kv, seq,
+                                                  chunk, xscale, e, st);
 }
 
 }  // namespace dash

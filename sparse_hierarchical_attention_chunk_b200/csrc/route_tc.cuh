@@ -45,6 +45,10 @@ namespace dash {
 struct RouteTcParams {
   float* w;
   uint32_t* mask;
+  // estimate_diagonal: keys and learned queries of stage 0 (else unused)
+  const __nv_bfloat16* K;
+  const float* qbar;
+  int diag;
   int n_q, n_kv, seq, chunk, n_c, nw, kbar_rows, n_tiles, n_bg, pos_base;
   float xscale, e;
 };
@@ -84,6 +88,7 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_s;
   __shared__ float xch[2][2][3][128];           // [parity][column half][value][row]: partial sums
+  __shared__ float khat[NPOS][128];             // estimate_diagonal: the positions' diagonal summaries
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = prm.n_tiles - 1 - (int)(blockIdx.x / prm.n_bg);    // late (heavy) tiles first
@@ -209,7 +214,11 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
     const int pos = pos0 + pl;
     const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int c_base = half * 512;                       // first chunk of this thread's range
-    const int cols = SPLIT ? (half ? n_elig - 512 : 512) : n_elig;
+    // estimate_diagonal: the query's own chunk c_i is one more candidate,
+    // held in TMEM column c_i (right after the eligible ones; column
+    // c_i - 512 of the upper half with SPLIT), so every pass below includes it
+    const bool dg = prm.diag != 0 && n_elig > 0;
+    const int cols = SPLIT ? (half ? n_elig - 512 + (dg ? 1 : 0) : 512) : n_elig + (dg ? 1 : 0);
     const int nblk = (cols + 31) >> 5;                   // the row's blocks (warp-uniform)
     const int nb0 = (nblk + 1) >> 1;
     const int bk_lo = ch ? nb0 : 0, bk_hi = ch ? nblk : nb0;   // this thread's blocks
@@ -246,6 +255,36 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
       xpar ^= 1;
     };
     int blocks_written = 0;                              // 32-chunk blocks of w written
+    // estimate_diagonal: stage 0's summary of the keys each position may see
+    // in its own chunk (warp p, position p), then this row's scaled logit
+    // against it; computed while the logit MMAs run
+    float xd = -INFINITY;
+    if (dg) {
+      if (warp < NPOS)
+        summarize_chunk_warp<__nv_bfloat16, 128, 4, float>(
+            prm.K + ((size_t)bg * prm.seq + (size_t)c_i * prm.chunk) * 128, prm.qbar + g * 128,
+            khat[warp], pos0 + warp - c_i * prm.chunk + 1, lane);
+      rows_sync();
+      if (mbar_wait(&bar_q, 0, &abort_s)) {
+        // Q row (m & 63 with SPLIT: rows 64-127 repeat rows 0-63) from the
+        // 128-byte-swizzled tile, boxes 0 and 1 (columns 0-63, 64-127)
+        const int qr = SPLIT ? (m & 63) : m;
+        float acc = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          const uint8_t* qrow = sQ + kb * QBOX + (qr >> 3) * 1024 + (qr & 7) * 128;
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const uint4 v = *reinterpret_cast<const uint4*>(qrow + ((cc ^ (qr & 7)) << 4));
+            const __nv_bfloat16* qv = reinterpret_cast<const __nv_bfloat16*>(&v);
+            const float* kh = khat[pl] + kb * 64 + cc * 8;
+#pragma unroll
+            for (int e2 = 0; e2 < 8; ++e2) acc = fmaf(__bfloat162float(qv[e2]), kh[e2], acc);
+          }
+        }
+        xd = acc * prm.xscale;
+      }
+    }
     bool have = n_kt > 0 && mbar_wait(&bar_logits, 0, &abort_s);
     have = !rows_sync_or(!have);                         // all 256 threads agree
     if (have) {
@@ -262,9 +301,9 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
           const int cb = c_base + bk * 32;
 #pragma unroll
           for (int i = 0; i < 32; i += 2) f2_unpack(f2_mul(f2_pack(x[i], x[i + 1]), xs2), x[i], x[i + 1]);
-          if (cb + 32 > c_end) {                         // warp-uniform: the last block only
+          if (cb + 32 > c_end) {                         // warp-uniform: the last blocks only
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = cb + i < c_end ? x[i] : -INFINITY;
+            for (int i = 0; i < 32; ++i) x[i] = cb + i < c_end ? x[i] : (cb + i == c_i ? xd : -INFINITY);
           }
 #pragma unroll
           for (int i = 0; i < 32; i += 2) mx = fmax3(mx, x[i], x[i + 1]);
@@ -393,7 +432,9 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
             // aligned (the half-warp still writes one contiguous 128-byte span)
             if (c < prm.n_c) wrow[c] = w0;
             if (c + 1 < prm.n_c) wrow[c + 1] = w1;
-            uint32_t bits = ((w0 > 0.f ? 1u : 0u) | (w1 > 0.f ? 2u : 0u)) << (2 * h);
+            // the query's own chunk (estimate_diagonal) is never a mask bit
+            uint32_t bits = ((w0 > 0.f && c != c_i ? 1u : 0u) | (w1 > 0.f && c + 1 != c_i ? 2u : 0u))
+                            << (2 * h);
 #pragma unroll
             for (int sh = 1; sh < 16; sh <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, sh);
             if (h == 0) mrow[c0 >> 5] = bits;
@@ -421,6 +462,9 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
     for (int k = zfirst + (lane & 15); ch == 0 && k < zlast; k += 16) {
       mrow[k] = 0u;
       for (int i = 0; i < 32 && k * 32 + i < prm.n_c; ++i) wrow[k * 32 + i] = 0.f;
+      // estimate_diagonal on a row of the first chunk: the diagonal is the
+      // only candidate, weight 1
+      if (k == 0 && prm.diag && n_elig == 0) wrow[c_i] = 1.f;
     }
   }
   tc_fence_before();
@@ -470,9 +514,11 @@ cudaError_t launch_route_tc_part(const __nv_bfloat16* Q, const CUtensorMap& tk, 
   return launch_route_tc_k<SPLIT, kEntmaxGeneric>(tq, tk, prm, st);
 }
 
+// K, qbar: non-null for estimate_diagonal, else both null
 inline cudaError_t launch_route_tc(const __nv_bfloat16* Q, const __nv_bfloat16* Kbar, float* w,
-                                   uint32_t* mask, int batch, int n_q, int n_kv, int seq, int chunk,
-                                   float alpha, float gamma, cudaStream_t st) {
+                                   uint32_t* mask, const __nv_bfloat16* K, const float* qbar,
+                                   int batch, int n_q, int n_kv, int seq, int chunk, float alpha,
+                                   float gamma, cudaStream_t st) {
   const int n_c = (seq + chunk - 1) / chunk;
   CUtensorMap tk;
   {
@@ -484,6 +530,9 @@ inline cudaError_t launch_route_tc(const __nv_bfloat16* Q, const __nv_bfloat16* 
   RouteTcParams prm;
   prm.w = w;
   prm.mask = mask;
+  prm.K = K;
+  prm.qbar = qbar;
+  prm.diag = K != nullptr;
   prm.n_q = n_q;
   prm.n_kv = n_kv;
   prm.seq = seq;

@@ -17,13 +17,15 @@
 namespace dash {
 
 // One warp: the summary of the `chunk` rows at `base` (rows of D elements,
-// contiguous) with the learned query qh (D floats), written to dst (D elements).
+// contiguous) with the learned query qh (D floats), written to dst (D elements
+// of OutT: the keys' type for the summary cache, float for the estimated
+// summary of a partial chunk that routing uses without storing it).
 // UNROLL row groups are loaded per round; the rows are processed in the same
 // order whatever UNROLL is, so the result does not depend on it.
-template <typename T, int D, int UNROLL>
+template <typename T, int D, int UNROLL, typename OutT = T>
 __device__ __forceinline__ void summarize_chunk_warp(const T* __restrict__ base,
                                                      const float* __restrict__ qh,
-                                                     T* __restrict__ dst, int chunk, int lane) {
+                                                     OutT* __restrict__ dst, int chunk, int lane) {
   constexpr int EPV = 16 / sizeof(T);      // elements per 16-byte vector
   constexpr int LPR = D / EPV;             // lanes per row
   constexpr int RPW = 32 / LPR;            // rows per warp step
@@ -90,10 +92,15 @@ __device__ __forceinline__ void summarize_chunk_warp(const T* __restrict__ base,
     for (int e = 0; e < EPV; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
   if (grp == 0) {
     const float inv = 1.f / l;
-    T outv[EPV];
+    if constexpr (sizeof(OutT) == sizeof(T)) {
+      OutT outv[EPV];
 #pragma unroll
-    for (int e = 0; e < EPV; ++e) outv[e] = Elem<T>::from_f(acc[e] * inv);
-    *reinterpret_cast<uint4*>(dst + sub * EPV) = *reinterpret_cast<const uint4*>(outv);
+      for (int e = 0; e < EPV; ++e) outv[e] = Elem<OutT>::from_f(acc[e] * inv);
+      *reinterpret_cast<uint4*>(dst + sub * EPV) = *reinterpret_cast<const uint4*>(outv);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) dst[sub * EPV + e] = Elem<OutT>::from_f(acc[e] * inv);
+    }
   }
 }
 

@@ -53,6 +53,7 @@ class DashProblem(ctypes.Structure):
         ("gamma", ctypes.c_float),
         ("sigma", ctypes.c_float),
         ("dtype", ctypes.c_int32),
+        ("estimate_diagonal", ctypes.c_int32),
     ]
 
 
@@ -85,17 +86,18 @@ def lib():
         L.dash_attn_bwd.restype = i32
         L.dash_attn_bwd.argtypes = [P] + [vp] * 13
         L.dash_route.restype = i32
-        L.dash_route.argtypes = [P, vp, vp, vp, vp, vp]
+        L.dash_route.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.dash_attn_fwd.restype = i32
         L.dash_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.dash_workspace_bytes.restype = ctypes.c_size_t
         L.dash_workspace_bytes.argtypes = [P, i32]
         L.dash_decode.restype = i32
-        L.dash_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.dash_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.dash_decode_varlen.restype = i32
-        L.dash_decode_varlen.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.dash_decode_varlen.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                         ctypes.c_size_t, vp]
         L.dash_decode_paged.restype = i32
-        L.dash_decode_paged.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+        L.dash_decode_paged.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                         ctypes.c_size_t, vp]
         L.dash_selftest_wait_timeout.restype = i32
         L.dash_selftest_wait_timeout.argtypes = [vp]
@@ -114,15 +116,17 @@ def status_str(status):
 
 
 def problem(batch, n_q_heads, n_kv_heads, seq_len, head_dim, chunk, alpha=1.5, gamma=1.0,
-            sigma=1.0, dtype="bf16"):
+            sigma=1.0, dtype="bf16", estimate_diagonal=False):
     return DashProblem(batch, n_q_heads, n_kv_heads, seq_len, head_dim, chunk, alpha, gamma, sigma,
-                       DASH_BF16 if dtype in ("bf16", torch.bfloat16) else DASH_F32)
+                       DASH_BF16 if dtype in ("bf16", torch.bfloat16) else DASH_F32,
+                       1 if estimate_diagonal else 0)
 
 
-def problem_for(wl, sigma=None):
+def problem_for(wl, sigma=None, estimate_diagonal=False):
     """DashProblem for a :class:`configs.Workload`."""
     return problem(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.seq, wl.head_dim, wl.chunk,
-                   wl.alpha, wl.gamma, wl.sigma if sigma is None else sigma, wl.dtype)
+                   wl.alpha, wl.gamma, wl.sigma if sigma is None else sigma, wl.dtype,
+                   estimate_diagonal)
 
 
 def _tdtype(p):
@@ -269,14 +273,21 @@ def backward(p, Q, K, V, qbar, out, dO, stream=None):
     return {"dQ": dQ, "dK": dK, "dV": dV, "dqbar": dqbar, "dw": dw, "dKbar": dKbar}
 
 
-def dash_route(p, Q, Kbar, w, mask, stream=None):
+def dash_route(p, Q, Kbar, w, mask, stream=None, K=None, qbar=None):
+    """Stage 1; with p.estimate_diagonal the keys K and learned queries qbar
+    of stage 0 are required as well."""
     dt = _tdtype(p)
     _check(Q, "Q", (p.batch, p.n_q_heads, p.seq_len, p.head_dim), dt)
     _check(Kbar, "Kbar", (p.batch, p.n_kv_heads, p.seq_len // p.chunk, p.head_dim), dt)
     _check(w, "w", (p.batch, p.n_kv_heads, p.seq_len, n_chunks(p)), torch.float32)
     _check(mask, "mask", (p.batch, p.n_kv_heads, p.seq_len, n_words(p)), torch.int32)
-    _raise("dash_route", lib().dash_route(ctypes.byref(p), _ptr(Q), _ptr(Kbar), _ptr(w), _ptr(mask),
-                                          _stream(stream)))
+    if p.estimate_diagonal:
+        if K is None or qbar is None:
+            raise ValueError("estimate_diagonal needs K and qbar")
+        _check(K, "K", (p.batch, p.n_kv_heads, p.seq_len, p.head_dim), dt)
+        _check(qbar, "qbar", (p.n_kv_heads, p.head_dim), torch.float32)
+    _raise("dash_route", lib().dash_route(ctypes.byref(p), _ptr(Q), _ptr(Kbar), _ptr(K), _ptr(qbar),
+                                          _ptr(w), _ptr(mask), _stream(stream)))
 
 
 def dash_workspace_bytes(p, is_decode):
@@ -300,11 +311,11 @@ def dash_attn_fwd(p, Q, K, V, w, mask, O, lse=None, workspace=None, stream=None)
 
 
 def dash_decode(p, q, Kc, Vc, Kbar, o, lse=None, w=None, mask=None, workspace=None, stream=None,
-                cache_lens=None, page_table=None):
+                cache_lens=None, page_table=None, qbar=None):
     """One decode step; with cache_lens (int32 [batch] on the device) each
     sequence has its own length and p.seq_len is the caches' capacity; with
     page_table (int32 [batch, max_pages]) as well, Kc and Vc are page pools
-    [n_pages, n_kv_heads, chunk, head_dim]."""
+    [n_pages, n_kv_heads, chunk, head_dim].  p.estimate_diagonal needs qbar."""
     dt = _tdtype(p)
     L = p.seq_len
     _check(q, "q", (p.batch, p.n_q_heads, p.head_dim), dt)
@@ -326,12 +337,16 @@ def dash_decode(p, q, Kc, Vc, Kbar, o, lse=None, w=None, mask=None, workspace=No
         _check(w, "w", (p.batch, p.n_kv_heads, n_chunks(p)), torch.float32)
     if mask is not None:
         _check(mask, "mask", (p.batch, p.n_kv_heads, n_words(p)), torch.int32)
+    if p.estimate_diagonal:
+        if qbar is None:
+            raise ValueError("estimate_diagonal needs qbar")
+        _check(qbar, "qbar", (p.n_kv_heads, p.head_dim), torch.float32)
     if workspace is None:
         workspace = torch.empty(dash_workspace_bytes(p, True), dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     if cache_lens is None:
         _raise("dash_decode", lib().dash_decode(ctypes.byref(p), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Kbar),
-                                                _ptr(o), _ptr(lse), _ptr(w), _ptr(mask),
+                                                _ptr(qbar), _ptr(o), _ptr(lse), _ptr(w), _ptr(mask),
                                                 _ptr(workspace), ws_bytes, _stream(stream)))
         return
     _check(cache_lens, "cache_lens", (p.batch,), torch.int32)
@@ -339,24 +354,25 @@ def dash_decode(p, q, Kc, Vc, Kbar, o, lse=None, w=None, mask=None, workspace=No
         _raise("dash_decode_paged",
                lib().dash_decode_paged(ctypes.byref(p), _ptr(cache_lens), _ptr(page_table),
                                        int(page_table.shape[1]), int(Kc.shape[0]), _ptr(q), _ptr(Kc),
-                                       _ptr(Vc), _ptr(Kbar), _ptr(o), _ptr(lse), _ptr(w), _ptr(mask),
-                                       _ptr(workspace), ws_bytes, _stream(stream)))
+                                       _ptr(Vc), _ptr(Kbar), _ptr(qbar), _ptr(o), _ptr(lse), _ptr(w),
+                                       _ptr(mask), _ptr(workspace), ws_bytes, _stream(stream)))
         return
     _raise("dash_decode_varlen",
            lib().dash_decode_varlen(ctypes.byref(p), _ptr(cache_lens), _ptr(q), _ptr(Kc), _ptr(Vc),
-                                    _ptr(Kbar), _ptr(o), _ptr(lse), _ptr(w), _ptr(mask),
+                                    _ptr(Kbar), _ptr(qbar), _ptr(o), _ptr(lse), _ptr(w), _ptr(mask),
                                     _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def dash_decode_varlen(p, cache_lens, q, Kc, Vc, Kbar, o, lse=None, w=None, mask=None,
-                       workspace=None, stream=None):
-    dash_decode(p, q, Kc, Vc, Kbar, o, lse, w, mask, workspace, stream, cache_lens=cache_lens)
+                       workspace=None, stream=None, qbar=None):
+    dash_decode(p, q, Kc, Vc, Kbar, o, lse, w, mask, workspace, stream, cache_lens=cache_lens,
+                qbar=qbar)
 
 
 def dash_decode_paged(p, cache_lens, page_table, q, Kpool, Vpool, Kbar, o, lse=None, w=None,
-                      mask=None, workspace=None, stream=None):
+                      mask=None, workspace=None, stream=None, qbar=None):
     dash_decode(p, q, Kpool, Vpool, Kbar, o, lse, w, mask, workspace, stream,
-                cache_lens=cache_lens, page_table=page_table)
+                cache_lens=cache_lens, page_table=page_table, qbar=qbar)
 
 
 def dash_decode_noalloc(p, q, Kc, Vc, Kbar, o, lse=None, w=None, mask=None, stream=None):
@@ -428,7 +444,7 @@ def prefill(p, Q, K, V, qbar, out=None, stream=None, with_lse=True):
     """Stage 0 -> stage 1 -> stage 2 on the device; returns the output dict."""
     out = alloc_prefill(p, Q.device) if out is None else out
     dash_summarize(p, K, qbar, out["Kbar"], stream=stream)
-    dash_route(p, Q, out["Kbar"], out["w"], out["mask"], stream=stream)
+    dash_route(p, Q, out["Kbar"], out["w"], out["mask"], stream=stream, K=K, qbar=qbar)
     dash_attn_fwd(p, Q, K, V, out["w"], out["mask"], out["O"], out["lse"] if with_lse else None,
                   stream=stream)
     return out
@@ -445,8 +461,9 @@ def alloc_decode(p, device="cuda"):
     }
 
 
-def decode(p, q, Kc, Vc, Kbar, out=None, stream=None, cache_lens=None, page_table=None):
+def decode(p, q, Kc, Vc, Kbar, out=None, stream=None, cache_lens=None, page_table=None,
+           qbar=None):
     out = alloc_decode(p, q.device) if out is None else out
     dash_decode(p, q, Kc, Vc, Kbar, out["o"], out["lse"], out["w"], out["mask"], out["workspace"],
-                stream=stream, cache_lens=cache_lens, page_table=page_table)
+                stream=stream, cache_lens=cache_lens, page_table=page_table, qbar=qbar)
     return out

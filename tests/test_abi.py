@@ -38,7 +38,7 @@ def test_status_strings_and_version(L):
     assert dash.status_str(0) == "DASH_OK"
     assert dash.status_str(4) == "DASH_ERR_TIMEOUT"
     assert dash.status_str(99) == "DASH_ERR_UNKNOWN"
-    assert L.dash_version() >> 16 == 1
+    assert L.dash_version() >> 16 == 2
 
 
 def _p(**kw):
@@ -65,17 +65,17 @@ host_only = pytest.mark.skipif(__import__("torch").cuda.is_available(),
 @host_only
 def test_invalid_problem_rejected(L, kw):
     p = _p(**kw)
-    st = L.dash_route(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None)
+    st = L.dash_route(ctypes.byref(p), FAKE, FAKE, None, None, FAKE, FAKE, None)
     assert st == dash.DASH_ERR_INVALID_ARG
 
 
 @host_only
 def test_null_and_misaligned_pointers_rejected(L):
     p = _p()
-    assert L.dash_route(None, FAKE, FAKE, FAKE, FAKE, None) == dash.DASH_ERR_INVALID_ARG
-    assert L.dash_route(ctypes.byref(p), None, FAKE, FAKE, FAKE, None) == dash.DASH_ERR_INVALID_ARG
+    assert L.dash_route(None, FAKE, FAKE, None, None, FAKE, FAKE, None) == dash.DASH_ERR_INVALID_ARG
+    assert L.dash_route(ctypes.byref(p), None, FAKE, None, None, FAKE, FAKE, None) == dash.DASH_ERR_INVALID_ARG
     odd = ctypes.c_void_p((1 << 20) + 8)
-    assert L.dash_route(ctypes.byref(p), odd, FAKE, FAKE, FAKE, None) == dash.DASH_ERR_INVALID_ARG
+    assert L.dash_route(ctypes.byref(p), odd, FAKE, None, None, FAKE, FAKE, None) == dash.DASH_ERR_INVALID_ARG
     assert L.dash_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 0,
                            None) == dash.DASH_ERR_INVALID_ARG
     assert L.dash_summarize(ctypes.byref(p), FAKE, FAKE, 0, 17, FAKE, None) == dash.DASH_ERR_INVALID_ARG
@@ -90,28 +90,28 @@ def test_unsupported_shapes(L):
                            None) == dash.DASH_ERR_UNSUPPORTED
     # routing keeps a row of chunk scores per warp in registers: n_c <= 2048
     p = _p(seq_len=2048 * 64 + 64)
-    assert L.dash_route(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None) == dash.DASH_ERR_UNSUPPORTED
+    assert L.dash_route(ctypes.byref(p), FAKE, FAKE, None, None, FAKE, FAKE, None) == dash.DASH_ERR_UNSUPPORTED
     # decode runs in bf16
     p = _p(dtype="f32", seq_len=1000)
-    assert L.dash_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE,
-                         1 << 30, None) == dash.DASH_ERR_UNSUPPORTED
+    assert L.dash_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, None,
+                         FAKE, 1 << 30, None) == dash.DASH_ERR_UNSUPPORTED
 
 
 @host_only
 def test_decode_varlen_lengths_pointer_checked(L):
     p = _p(batch=8, seq_len=131072)
     need = dash.dash_workspace_bytes(p, True)
-    assert L.dash_decode_varlen(ctypes.byref(p), None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
-                                FAKE, need, None) == dash.DASH_ERR_INVALID_ARG
+    assert L.dash_decode_varlen(ctypes.byref(p), None, FAKE, FAKE, FAKE, FAKE, None, FAKE, None,
+                                None, None, FAKE, need, None) == dash.DASH_ERR_INVALID_ARG
     odd = ctypes.c_void_p((1 << 20) + 2)
-    assert L.dash_decode_varlen(ctypes.byref(p), odd, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
-                                FAKE, need, None) == dash.DASH_ERR_INVALID_ARG
+    assert L.dash_decode_varlen(ctypes.byref(p), odd, FAKE, FAKE, FAKE, FAKE, None, FAKE, None,
+                                None, None, FAKE, need, None) == dash.DASH_ERR_INVALID_ARG
     # the rest is dash_decode's validation
-    assert L.dash_decode_varlen(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
-                                FAKE, need - 1, None) == dash.DASH_ERR_WORKSPACE
+    assert L.dash_decode_varlen(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None,
+                                None, None, FAKE, need - 1, None) == dash.DASH_ERR_WORKSPACE
     p = _p(dtype="f32", seq_len=1000)
-    assert L.dash_decode_varlen(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
-                                FAKE, 1 << 30, None) == dash.DASH_ERR_UNSUPPORTED
+    assert L.dash_decode_varlen(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None,
+                                None, None, FAKE, 1 << 30, None) == dash.DASH_ERR_UNSUPPORTED
 
 
 @host_only
@@ -120,8 +120,8 @@ def test_decode_paged_arguments_checked(L):
     need = dash.dash_workspace_bytes(p, True)
     n_c = 131072 // 64
     args = lambda lens, table, max_pages, n_pages: (ctypes.byref(p), lens, table, max_pages, n_pages,
-                                                    FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
-                                                    FAKE, need, None)
+                                                    FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None,
+                                                    None, FAKE, need, None)
     odd = ctypes.c_void_p((1 << 20) + 2)
     assert L.dash_decode_paged(*args(None, FAKE, n_c, 10)) == dash.DASH_ERR_INVALID_ARG
     assert L.dash_decode_paged(*args(FAKE, None, n_c, 10)) == dash.DASH_ERR_INVALID_ARG
@@ -158,7 +158,37 @@ def test_decode_workspace_checked(L):
     need = dash.dash_workspace_bytes(p, True)
     assert need > 0 and need % 256 == 0
     assert dash.dash_workspace_bytes(p, False) == 0
-    assert L.dash_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE,
-                         need - 1, None) == dash.DASH_ERR_WORKSPACE
-    assert L.dash_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, None,
-                         need, None) == dash.DASH_ERR_WORKSPACE
+    assert L.dash_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, None,
+                         FAKE, need - 1, None) == dash.DASH_ERR_WORKSPACE
+    assert L.dash_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, None,
+                         None, need, None) == dash.DASH_ERR_WORKSPACE
+
+
+@host_only
+def test_estimate_diagonal_arguments_checked(L):
+    # the flag is 0 or 1; with it, routing needs K and qbar, decode needs qbar
+    p = _p()
+    p.estimate_diagonal = 2
+    assert L.dash_route(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == \
+        dash.DASH_ERR_INVALID_ARG
+    p.estimate_diagonal = 1
+    assert L.dash_route(ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == \
+        dash.DASH_ERR_INVALID_ARG
+    assert L.dash_route(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE, FAKE, None) == \
+        dash.DASH_ERR_INVALID_ARG
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert L.dash_route(ctypes.byref(p), FAKE, FAKE, odd, FAKE, FAKE, FAKE, None) == \
+        dash.DASH_ERR_INVALID_ARG
+    # no entmax normalisation in top-k routing, no gradient through the
+    # diagonal candidate, no qbar argument in the no-allocation decode
+    assert L.dash_route_topk(ctypes.byref(p), FAKE, FAKE, 4, FAKE, FAKE, None) == \
+        dash.DASH_ERR_UNSUPPORTED
+    assert L.dash_route_bwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None) == \
+        dash.DASH_ERR_UNSUPPORTED
+    pd = _p(batch=8, seq_len=131072)
+    pd.estimate_diagonal = 1
+    need = dash.dash_workspace_bytes(pd, True)
+    assert L.dash_decode(ctypes.byref(pd), FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, None,
+                         FAKE, need, None) == dash.DASH_ERR_INVALID_ARG
+    assert L.dash_decode_noalloc(ctypes.byref(pd), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
+                                 None) == dash.DASH_ERR_UNSUPPORTED

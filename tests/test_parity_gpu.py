@@ -106,16 +106,17 @@ def test_summarize_partial_range_appends():
 # stage 1
 # ----------------------------------------------------------------------------
 
-def _route_case(wl, seed, positions=None):
+def _route_case(wl, seed, positions=None, diag=False):
     inp = synth.make_prefill(wl, seed=seed)
     kb = oracle_kbar(inp["K"], inp["qbar"], wl.chunk, _dt(wl))
-    p = dash.problem_for(wl)
+    p = dash.problem_for(wl, estimate_diagonal=diag)
     n_c = wl.n_chunks
     w = torch.empty(wl.batch, wl.n_kv_heads, wl.seq, n_c, device="cuda")
     mask = torch.empty(wl.batch, wl.n_kv_heads, wl.seq, (n_c + 31) // 32, dtype=torch.int32, device="cuda")
-    dash.dash_route(p, inp["Q"].cuda(), kb.cuda(), w, mask)
+    dash.dash_route(p, inp["Q"].cuda(), kb.cuda(), w, mask, K=inp["K"].cuda(), qbar=inp["qbar"].cuda())
     torch.cuda.synchronize()
-    wr, mr, near = oracle.route(inp["Q"], kb, wl.alpha, wl.gamma, wl.chunk, positions=positions)
+    wr, mr, near = oracle.route(inp["Q"], kb, wl.alpha, wl.gamma, wl.chunk, positions=positions,
+                                diag=(inp["K"], inp["qbar"]) if diag else None)
     pos = slice(None) if positions is None else positions
     wg = np64(w)[:, :, pos]
     mg = mask_from_dev(mask)[:, :, pos]
@@ -143,6 +144,41 @@ def test_route_more_than_512_chunks_sampled():
     n_diff, n_bad = compare_masks(mg, mr, near, wl.n_chunks)
     assert n_bad == 0, f"{n_bad} mask bits differ away from tau ({n_diff} total)"
     assert np.abs(wg - wr).max() <= TOL_W
+
+
+@pytest.mark.parametrize("name", list(MED))
+def test_route_estimate_diagonal_matches_oracle(name):
+    # the query's own chunk as one more entmax candidate (tensor-core routing
+    # for the G = 16, d = 128 cases, the generic kernel for the others)
+    wl = MED[name]
+    wg, mg, wr, mr, near = _route_case(wl, seed=31, diag=True)
+    n_diff, n_bad = compare_masks(mg, mr, near, wl.n_chunks)
+    print(f"near-threshold mask flips: {n_diff}")
+    assert n_bad == 0, f"{n_bad} mask bits differ away from tau ({n_diff} total)"
+    assert np.abs(wg - wr).max() <= TOL_W
+    # the diagonal's weight is reported in column c_i; rows of the first chunk give it 1
+    c_i = np.arange(wl.seq) // wl.chunk
+    wd = np.take_along_axis(wg, c_i[None, None, :, None], axis=-1)[..., 0]
+    assert np.allclose(wd[:, :, :wl.chunk], 1.0)
+    assert np.any((wd > 0) & (wd < 1))                  # the candidate really competes
+
+
+def test_route_estimate_diagonal_more_than_512_chunks_sampled():
+    wl = W("med_split", "prefill", 1, 32, 2, 600 * 64, 128, 64, rho=(0.9, 0.2), needles=(3, 1))
+    pos = np.array([0, 63, 64, 100, 511 * 64 + 5, 511 * 64 + 63, 512 * 64, 513 * 64 + 17,
+                    530 * 64 + 63, 599 * 64, 600 * 64 - 1])
+    wg, mg, wr, mr, near = _route_case(wl, seed=32, positions=pos, diag=True)
+    n_diff, n_bad = compare_masks(mg, mr, near, wl.n_chunks)
+    assert n_bad == 0, f"{n_bad} mask bits differ away from tau ({n_diff} total)"
+    assert np.abs(wg - wr).max() <= TOL_W
+
+
+def test_route_estimate_diagonal_tiny_f32():
+    wl = configs.TINY_F32
+    wg, mg, wr, mr, near = _route_case(wl, seed=33, diag=True)
+    n_diff, n_bad = compare_masks(mg, mr, near, wl.n_chunks)
+    assert n_bad == 0
+    assert np.abs(wg - wr).max() <= 1e-5
 
 
 def test_route_tiny_f32():
@@ -257,6 +293,26 @@ def test_end_to_end_bf16():
     assert np.abs(np64(out["lse"]) - lr).max() <= TOL_LSE
 
 
+def test_end_to_end_estimate_diagonal_bf16():
+    # the chain with the diagonal candidate in the routing: every output,
+    # each stage on the GPU's own upstream result
+    wl = MED["g16_d128_b64_nc37"]
+    inp = synth.make_prefill(wl, seed=37)
+    p = dash.problem_for(wl, estimate_diagonal=True)
+    out = dash.prefill(p, inp["Q"].cuda(), inp["K"].cuda(), inp["V"].cuda(), inp["qbar"].cuda())
+    torch.cuda.synchronize()
+    wr, mr, near = oracle.route(inp["Q"], out["Kbar"].cpu(), wl.alpha, wl.gamma, wl.chunk,
+                                diag=(inp["K"], inp["qbar"]))
+    mg = mask_from_dev(out["mask"])
+    n_diff, n_bad = compare_masks(mg, mr, near, wl.n_chunks)
+    assert n_bad == 0
+    wg = np64(out["w"])
+    assert np.abs(wg - wr).max() <= TOL_W
+    Or, lr = oracle.attn_fwd(inp["Q"], inp["K"], inp["V"], wg, mg, wl.sigma, wl.chunk)
+    assert np.abs(np64(out["O"]) - Or).max() <= TOL_O_BF16
+    assert np.abs(np64(out["lse"]) - lr).max() <= TOL_LSE
+
+
 # ----------------------------------------------------------------------------
 # full-size workloads: sampled rows (rows are independent given K, V, Kbar)
 # ----------------------------------------------------------------------------
@@ -334,15 +390,16 @@ DEC = {
 }
 
 
-def _decode_case(wl, seed):
+def _decode_case(wl, seed, diag=False):
     inp = synth.make_decode(wl, seed=seed)
     kb = oracle_kbar(inp["K"], inp["qbar"], wl.chunk, torch.bfloat16) if wl.seq >= wl.chunk else \
         torch.zeros(wl.batch, wl.n_kv_heads, 0, wl.head_dim, dtype=torch.bfloat16)
-    p = dash.problem_for(wl)
-    out = dash.decode(p, inp["q"].cuda(), inp["K"].cuda(), inp["V"].cuda(), kb.cuda())
+    p = dash.problem_for(wl, estimate_diagonal=diag)
+    out = dash.decode(p, inp["q"].cuda(), inp["K"].cuda(), inp["V"].cuda(), kb.cuda(),
+                      qbar=inp["qbar"].cuda())
     assert dash.dash_get_error() == dash.DASH_OK
     ref = oracle.decode(inp["q"], inp["K"], inp["V"], kb, wl.seq, wl.alpha, wl.gamma, wl.sigma,
-                        wl.chunk)
+                        wl.chunk, qbar=inp["qbar"] if diag else None)
     return out, ref, inp, kb
 
 
@@ -352,6 +409,15 @@ def test_decode_matches_oracle(name):
     out, ref, inp, kb = _decode_case(wl, seed=12)
     if name.endswith("_dense"):                    # the case must really be dense
         assert (np64(out["w"])[..., : (wl.seq - 1) // wl.chunk] > 0).all()
+    _check_decode(wl, out, ref, inp["q"], inp["K"], inp["V"], None)
+
+
+@pytest.mark.parametrize("name", ["b2_L1000_ragged", "b3_L64_first_chunk", "b1_L4097_b128_g8",
+                                  "b4_L3000_d64_g4", "b2_L2000_alpha13",
+                                  "b2_L5000_b128_sparsemax_sigma0"])
+def test_decode_estimate_diagonal_matches_oracle(name):
+    wl = DEC[name]
+    out, ref, inp, kb = _decode_case(wl, seed=34, diag=True)
     _check_decode(wl, out, ref, inp["q"], inp["K"], inp["V"], None)
 
 
@@ -393,16 +459,16 @@ DECV = {
 }
 
 
-def _decode_varlen_case(wl, lens, seed):
+def _decode_varlen_case(wl, lens, seed, diag=False):
     inp = synth.make_decode(wl, seed=seed)
     lens = inp["lens"] if lens is None else torch.tensor(lens, dtype=torch.int32)
     kb = oracle_kbar(inp["K"], inp["qbar"], wl.chunk, torch.bfloat16)
-    p = dash.problem_for(wl)
+    p = dash.problem_for(wl, estimate_diagonal=diag)
     out = dash.decode(p, inp["q"].cuda(), inp["K"].cuda(), inp["V"].cuda(), kb.cuda(),
-                      cache_lens=lens.cuda())
+                      cache_lens=lens.cuda(), qbar=inp["qbar"].cuda())
     assert dash.dash_get_error() == dash.DASH_OK
     ref = oracle.decode_varlen(inp["q"], inp["K"], inp["V"], kb, lens.tolist(), wl.alpha, wl.gamma,
-                               wl.sigma, wl.chunk)
+                               wl.sigma, wl.chunk, qbar=inp["qbar"] if diag else None)
     return out, ref, lens, inp
 
 
@@ -435,6 +501,13 @@ def _check_decode(wl, out, ref, q, Kc, Vc, lens):
 def test_decode_varlen_matches_oracle(name):
     wl, lens = DECV[name]
     out, ref, lens, inp = _decode_varlen_case(wl, lens, seed=14)
+    _check_decode(wl, out, ref, inp["q"], inp["K"], inp["V"], lens.tolist())
+
+
+@pytest.mark.parametrize("name", list(DECV))
+def test_decode_varlen_estimate_diagonal_matches_oracle(name):
+    wl, lens = DECV[name]
+    out, ref, lens, inp = _decode_varlen_case(wl, lens, seed=35, diag=True)
     _check_decode(wl, out, ref, inp["q"], inp["K"], inp["V"], lens.tolist())
 
 
@@ -498,18 +571,18 @@ def test_decode_varlen_length_out_of_range_is_reported():
 # decode over paged caches
 # ----------------------------------------------------------------------------
 
-def _decode_paged_case(wl, lens, seed, extra_pages=7):
+def _decode_paged_case(wl, lens, seed, extra_pages=7, diag=False):
     inp = synth.make_decode(wl, seed=seed)
     lens = inp["lens"] if lens is None else torch.tensor(lens, dtype=torch.int32)
     kb = oracle_kbar(inp["K"], inp["qbar"], wl.chunk, torch.bfloat16)
     Kp, Vp, table = synth.to_pages(inp["K"], inp["V"], lens.tolist(), wl.chunk, seed=seed,
                                    extra_pages=extra_pages)
-    p = dash.problem_for(wl)
+    p = dash.problem_for(wl, estimate_diagonal=diag)
     out = dash.decode(p, inp["q"].cuda(), Kp.cuda(), Vp.cuda(), kb.cuda(), cache_lens=lens.cuda(),
-                      page_table=table.cuda())
+                      page_table=table.cuda(), qbar=inp["qbar"].cuda())
     assert dash.dash_get_error() == dash.DASH_OK
     ref = oracle.decode_paged(inp["q"], Kp, Vp, kb, lens.tolist(), table.numpy(), wl.alpha,
-                              wl.gamma, wl.sigma, wl.chunk)
+                              wl.gamma, wl.sigma, wl.chunk, qbar=inp["qbar"] if diag else None)
     Kc, Vc = oracle.gather_pages(Kp, Vp, lens.tolist(), table.numpy(), wl.chunk)
     return out, ref, (inp["q"], Kc, Vc, lens.tolist())
 
@@ -518,6 +591,13 @@ def _decode_paged_case(wl, lens, seed, extra_pages=7):
 def test_decode_paged_matches_oracle(name):
     wl, lens = DECV[name]
     out, ref, (q, Kc, Vc, lens) = _decode_paged_case(wl, lens, seed=18)
+    _check_decode(wl, out, ref, q, Kc, Vc, lens)
+
+
+@pytest.mark.parametrize("name", list(DECV))
+def test_decode_paged_estimate_diagonal_matches_oracle(name):
+    wl, lens = DECV[name]
+    out, ref, (q, Kc, Vc, lens) = _decode_paged_case(wl, lens, seed=36, diag=True)
     _check_decode(wl, out, ref, q, Kc, Vc, lens)
 
 
