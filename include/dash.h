@@ -144,6 +144,28 @@ int dash_route(const dash_problem* p, const void* Q, const void* Kbar, const voi
                const float* qbar, float* w, uint32_t* mask, void* stream);
 
 /*
+ * Stage 1 with its weights in compact form: for each row, only the routed
+ * chunks, in increasing chunk order (gist.science summary, Fase 2
+ * "Implementatie": the attention kernel walks the active chunks of a
+ * bit-packed mask and adds the routing bias).  Same routing as dash_route
+ * (estimate_diagonal included; the query's own chunk is not a routed
+ * chunk and is not listed); instead of the dense w it writes
+ *   mask   [b, Hkv, N, n_w] uint32, as dash_route;
+ *   weight [b, Hkv, N, n_c] float: entry k of a row is the weight of the
+ *          chunk of the k-th set bit of the row's mask;
+ *   count  [b, Hkv, N] int32 (nullable): the number of set bits of the row;
+ *   index  [b, Hkv, N, n_c] int32 (nullable): entry k is that chunk.
+ * Only the first count entries of a row of weight and index are written;
+ * the rest of the row is left as it was.  A row's bytes written are thus
+ * proportional to its support, not to n_c.  dash_attn_fwd_packed reads
+ * (weight, mask).  Errors: as dash_route (count/index misaligned ->
+ * DASH_ERR_INVALID_ARG).
+ */
+int dash_route_packed(const dash_problem* p, const void* Q, const void* Kbar, const void* K,
+                      const float* qbar, uint32_t* mask, int32_t* count, int32_t* index,
+                      float* weight, void* stream);
+
+/*
  * Fixed-budget top-k routing on the same summaries: the baseline the pages
  * contrast with (gist.science summary, "Probleemstelling": NSA and
  * InfLLMv2 select the top-k KV blocks by coarse attention scores, then run
@@ -234,6 +256,17 @@ int dash_route_bwd(const dash_problem* p, const void* Q, const void* Kbar, const
  */
 int dash_summarize_bwd(const dash_problem* p, const void* K, const float* qbar, const float* dKbar,
                        float* dK, float* dqbar, void* stream);
+
+/*
+ * dash_attn_fwd on the compact weights of dash_route_packed: `weight` holds,
+ * per row, the weights of the row's routed chunks in increasing chunk order
+ * (entry k belongs to the k-th set bit of the row's mask); the entries past
+ * a row's count are never used.  Same output, errors and limits as
+ * dash_attn_fwd.
+ */
+int dash_attn_fwd_packed(const dash_problem* p, const void* Q, const void* K, const void* V,
+                         const float* weight, const uint32_t* mask, void* O, float* lse,
+                         void* stream);
 
 /* Workspace bytes needed by dash_attn_fwd (is_decode = 0) or dash_decode (1). */
 size_t dash_workspace_bytes(const dash_problem* p, int is_decode);

@@ -29,6 +29,8 @@ from .dash_oracle import (  # noqa: F401
     route,
     route_topk,
     pack_mask,
+    pack_weights,
+    unpack_weights,
     unpack_mask,
     attn_fwd,
     decode,

@@ -97,6 +97,11 @@ What pins each function (``tests/test_oracle.py``):
   cache rebuilds ``chunk_summary`` of the whole cache; rows of sequences not
   at a boundary are left as they were; the paged form equals the contiguous
   one through an identity table.
+* ``pack_weights`` / ``unpack_weights`` (the compact routing form): on
+  ``route``'s output the round trip returns the dense w and the mask; counts
+  are the popcounts of the mask rows; indices ascend and are the set bits;
+  each listed weight is the dense w at that chunk (checked element by
+  element against a direct scan of the dense rows).
 * ``decode_attend`` (stage 2 of a decode step on given routing): with every
   chunk active and w = 1 it is torch's SDPA of each query against its first
   L keys; on ``decode``'s own routing it returns ``decode``'s output; with one
@@ -229,6 +234,51 @@ def unpack_mask(words, n_c):
     for c in range(n_c):
         out[..., c] = ((words[..., c // 32] >> np.uint64(c % 32)) & np.uint64(1)) == 1
     return out
+
+
+def pack_weights(w, mask):
+    """Compact form of stage 1's output (gist.science summary, Fase 2
+    "Implementatie": stage 2 walks the active chunks of a bit-packed mask).
+
+    For every row, the chunks whose mask bit is set, in increasing order, and
+    their weights: returns (count [...] int32, index [..., n_c] int32,
+    weight [..., n_c] fp64), where only the first count entries of a row of
+    index and weight are meaningful (the rest are -1 and 0).
+    """
+    w = _f64(w)
+    n_c = w.shape[-1]
+    act = unpack_mask(mask, n_c)
+    count = act.sum(axis=-1).astype(np.int32)
+    index = np.full(w.shape, -1, dtype=np.int32)
+    weight = np.zeros(w.shape)
+    flat_a = act.reshape(-1, n_c)
+    flat_w = w.reshape(-1, n_c)
+    fi = index.reshape(-1, n_c)
+    fw = weight.reshape(-1, n_c)
+    for r in range(flat_a.shape[0]):
+        cs = np.nonzero(flat_a[r])[0]
+        fi[r, :cs.size] = cs
+        fw[r, :cs.size] = flat_w[r, cs]
+    return count, index, weight
+
+
+def unpack_weights(count, index, weight, n_c):
+    """Dense [..., n_c] weights (zero off the listed chunks) and the packed
+    mask from the compact form of ``pack_weights``."""
+    count = np.asarray(count)
+    index = np.asarray(index)
+    weight = _f64(weight)
+    dense = np.zeros(count.shape + (n_c,))
+    fd = dense.reshape(-1, n_c)
+    fc, fi, fw = count.reshape(-1), index.reshape(-1, index.shape[-1]), weight.reshape(-1, weight.shape[-1])
+    for r in range(fc.size):
+        k = int(fc[r])
+        fd[r, fi[r, :k]] = fw[r, :k]
+    act = np.zeros(dense.shape, dtype=bool)
+    fa = act.reshape(-1, n_c)
+    for r in range(fc.size):
+        fa[r, fi[r, :int(fc[r])]] = True
+    return dense, pack_mask(act)
 
 
 # ----------------------------------------------------------------------------

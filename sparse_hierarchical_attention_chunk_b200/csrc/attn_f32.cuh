@@ -12,7 +12,9 @@
 
 namespace dash {
 
-template <int D>
+// PACKED: w is the compact form of stage 1 (per row, the weights of the
+// routed chunks in increasing chunk order), else dense [rows][n_c].
+template <int D, bool PACKED>
 __global__ void __launch_bounds__(256) attn_f32_kernel(
     const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
     const float* __restrict__ w, const uint32_t* __restrict__ mask, float* __restrict__ O,
@@ -57,9 +59,11 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(
     m = m_new;
   };
   for (int j = c_i * chunk; j <= i; ++j) visit(j, 0.f);          // diagonal branch first
+  int rank = 0;                                                   // routed chunks seen so far
   for (int c = 0; c < c_i && c < n_c; ++c) {
     if (!((mrow[c >> 5] >> (c & 31)) & 1u)) continue;
-    const float bias = sigma == 0.f ? 0.f : sigma * log2f(wrow[c]);
+    const float wc = PACKED ? wrow[rank++] : wrow[c];
+    const float bias = sigma == 0.f ? 0.f : sigma * log2f(wc);
     if (bias == -INFINITY) continue;
     for (int j = c * chunk; j < (c + 1) * chunk; ++j) visit(j, bias);
   }
@@ -72,14 +76,19 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(
 template <int D>
 cudaError_t launch_attn_f32(const float* Q, const float* K, const float* V, const float* w,
                             const uint32_t* mask, float* O, float* lse, int batch, int n_q,
-                            int n_kv, int seq, int chunk, float sigma, cudaStream_t st) {
+                            int n_kv, int seq, int chunk, float sigma, cudaStream_t st,
+                            bool packed = false) {
   const int n_c = (seq + chunk - 1) / chunk;
   const long long n_rows = (long long)batch * n_q * seq;
   const int threads = 256;
   const long long blocks = (n_rows * 32 + threads - 1) / threads;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  attn_f32_kernel<D><<<(unsigned)blocks, threads, 0, st>>>(Q, K, V, w, mask, O, lse, n_q, n_kv, seq,
-                                                          chunk, n_c, sigma, scale_log2, n_rows);
+  if (packed)
+    attn_f32_kernel<D, true><<<(unsigned)blocks, threads, 0, st>>>(
+        Q, K, V, w, mask, O, lse, n_q, n_kv, seq, chunk, n_c, sigma, scale_log2, n_rows);
+  else
+    attn_f32_kernel<D, false><<<(unsigned)blocks, threads, 0, st>>>(
+        Q, K, V, w, mask, O, lse, n_q, n_kv, seq, chunk, n_c, sigma, scale_log2, n_rows);
   return cudaGetLastError();
 }
 

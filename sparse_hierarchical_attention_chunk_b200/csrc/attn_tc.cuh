@@ -47,8 +47,11 @@
 namespace dash {
 
 struct AttnParams {
+  // w: dense [rows][n_c], or (packed != 0) the compact form of stage 1:
+  // per row the weights of its routed chunks in increasing chunk order
   const float* w;
   const uint32_t* mask;
+  int packed;
   __nv_bfloat16* O;
   float* lse;
   int n_q, n_kv, seq, chunk, n_c, nw, G, P, n_ctiles, n_bg;
@@ -153,7 +156,9 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
   uint8_t* code = reinterpret_cast<uint8_t*>(list + prm.n_c + 1);    // [n_c + 1], bit t: tile t active
   uint32_t* mrows = reinterpret_cast<uint32_t*>(
       (reinterpret_cast<uintptr_t>(code + prm.n_c + 1) + 15) & ~static_cast<uintptr_t>(15));
-  float* w_sm = reinterpret_cast<float*>(mrows + 2 * prm.P * prm.nw);   // [NS][2P]
+  // compact weights: set bits of each position's mask before each word
+  int* mpre = reinterpret_cast<int*>(mrows + 2 * prm.P * prm.nw);          // [2P][nw]
+  float* w_sm = reinterpret_cast<float*>(mpre + 2 * prm.P * prm.nw);       // [NS][2P]
   const int n_wl = min(2 * prm.P, 32);      // producer lanes that fetch w
 
   // Barriers.  Each tile has one S buffer, so every barrier below advances at
@@ -258,6 +263,17 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
       cnt_s[1] = cnt1;
     }
   }
+  if (prm.packed && warp >= 1 && warp < 8) {
+    // the rank of chunk c in position q's compact row is mpre[q][c / 32]
+    // plus the set bits of word c / 32 below c
+    for (int q = tid - 32; q < 2 * P; q += 224) {
+      int acc = 0;
+      for (int k = 0; k < prm.nw; ++k) {
+        mpre[q * prm.nw + k] = acc;
+        acc += __popc(mrows[q * prm.nw + k]);
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -330,8 +346,14 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
           tma_load_2d(sV + s * L::KV_BYTES + kb * L::KV_BOX, &tmV, &bar_v_full[s], kb * 64, krow);
       }
       if (lane < n_wl) {
-        for (int q = lane; q < 2 * P; q += 32)
-          cp_async_4(w_sm + s * 2 * P + q, prm.w + (row0 + q) * prm.n_c + c);
+        for (int q = lane; q < 2 * P; q += 32) {
+          // a position that does not route to c reads a neighbouring entry
+          // of its own row (never used: its bias is -inf)
+          const int col = prm.packed ? mpre[q * prm.nw + (c >> 5)] +
+                                           __popc(mrows[q * prm.nw + (c >> 5)] & ((1u << (c & 31)) - 1u))
+                                     : c;
+          cp_async_4(w_sm + s * 2 * P + q, prm.w + (row0 + q) * prm.n_c + col);
+        }
         cp_async_arrive_noinc(&bar_v_full[s]);
       }
       issued_v = j + 1;
@@ -641,7 +663,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
 template <int D>
 size_t attn_tc_smem_bytes(int n_c, int nw, int P) {
   using L = TcLayout<64, D>;
-  return (size_t)L::OFF_AUX + (size_t)(n_c + 1) * 5 + 16 + (size_t)2 * P * nw * 4 +
+  return (size_t)L::OFF_AUX + (size_t)(n_c + 1) * 5 + 16 + (size_t)2 * P * nw * 8 +
          (size_t)L::NS * 2 * P * 4 + 1024;
 }
 

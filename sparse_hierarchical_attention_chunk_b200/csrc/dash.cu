@@ -64,7 +64,8 @@ using dash::make_tmap;
 
 template <int CHUNK, int D>
 int run_attn_tc(const dash_problem* p, const void* Q, const void* K, const void* V,
-                const float* w, const uint32_t* mask, void* O, float* lse, cudaStream_t st) {
+                const float* w, const uint32_t* mask, void* O, float* lse, bool packed,
+                cudaStream_t st) {
   const int G = p->n_q_heads / p->n_kv_heads;
   const int P = 128 / G;
   const uint64_t d = (uint64_t)D;
@@ -87,6 +88,7 @@ int run_attn_tc(const dash_problem* p, const void* Q, const void* K, const void*
   dash::AttnParams prm;
   prm.w = w;
   prm.mask = mask;
+  prm.packed = packed ? 1 : 0;
   prm.O = static_cast<bf16*>(O);
   prm.lse = lse;
   prm.n_q = p->n_q_heads;
@@ -267,12 +269,17 @@ int dash_summarize_bwd(const dash_problem* p, const void* K, const float* qbar, 
   return cuda_status(e);
 }
 
-int dash_route(const dash_problem* p, const void* Q, const void* Kbar, const void* K,
-               const float* qbar, float* w, uint32_t* mask, void* stream) {
+}  // extern "C"
+
+// dash_route (dense w) and dash_route_packed (compact weights, optional
+// count / index)
+static int route_entry(const dash_problem* p, const void* Q, const void* Kbar, const void* K,
+                       const float* qbar, float* w, uint32_t* mask, bool packed, int32_t* count,
+                       int32_t* index, void* stream) {
   int rc = check_problem(p, false);
   if (rc) return rc;
   if (!Q || !Kbar || !w || !mask || !aligned16(Q) || !aligned16(Kbar) || !aligned16(w) ||
-      !aligned16(mask))
+      !aligned16(mask) || (count && !aligned16(count)) || (index && !aligned16(index)))
     return DASH_ERR_INVALID_ARG;
   if (p->estimate_diagonal && (!K || !qbar || !aligned16(K) || !aligned16(qbar)))
     return DASH_ERR_INVALID_ARG;
@@ -286,18 +293,33 @@ int dash_route(const dash_problem* p, const void* Q, const void* Kbar, const voi
 #define DASH_ROUTE(T, D)                                                                      \
   dash::launch_route<T, D>(static_cast<const T*>(Q), static_cast<const T*>(Kbar), w, mask,    \
                            static_cast<const T*>(K), qbar, p->batch, p->n_q_heads,            \
-                           p->n_kv_heads, p->seq_len, p->chunk, p->alpha, p->gamma, st)
+                           p->n_kv_heads, p->seq_len, p->chunk, p->alpha, p->gamma, st,       \
+                           packed, count, index)
   const int G = p->n_q_heads / p->n_kv_heads;
   if (p->dtype == DASH_BF16 && p->head_dim == 128 && G == 16 && n_chunks(p) <= 1024)
     e = dash::launch_route_tc(static_cast<const bf16*>(Q), static_cast<const bf16*>(Kbar), w, mask,
                               static_cast<const bf16*>(K), qbar, p->batch, p->n_q_heads,
-                              p->n_kv_heads, p->seq_len, p->chunk, p->alpha, p->gamma, st);
+                              p->n_kv_heads, p->seq_len, p->chunk, p->alpha, p->gamma, st, packed,
+                              count, index);
   else if (p->dtype == DASH_BF16)
     e = p->head_dim == 128 ? DASH_ROUTE(bf16, 128) : DASH_ROUTE(bf16, 64);
   else
     e = p->head_dim == 128 ? DASH_ROUTE(float, 128) : DASH_ROUTE(float, 64);
 #undef DASH_ROUTE
   return cuda_status(e);
+}
+
+extern "C" {
+
+int dash_route(const dash_problem* p, const void* Q, const void* Kbar, const void* K,
+               const float* qbar, float* w, uint32_t* mask, void* stream) {
+  return route_entry(p, Q, Kbar, K, qbar, w, mask, false, nullptr, nullptr, stream);
+}
+
+int dash_route_packed(const dash_problem* p, const void* Q, const void* Kbar, const void* K,
+                      const float* qbar, uint32_t* mask, int32_t* count, int32_t* index,
+                      float* weight, void* stream) {
+  return route_entry(p, Q, Kbar, K, qbar, weight, mask, true, count, index, stream);
 }
 
 size_t dash_workspace_bytes(const dash_problem* p, int is_decode) {
@@ -307,11 +329,12 @@ size_t dash_workspace_bytes(const dash_problem* p, int is_decode) {
                                       p->head_dim, p->chunk);
 }
 
-int dash_attn_fwd(const dash_problem* p, const void* Q, const void* K, const void* V,
-                  const float* w, const uint32_t* mask, void* O, float* lse, void* workspace,
-                  size_t workspace_bytes, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
+}  // extern "C"
+
+// dash_attn_fwd (dense w) and dash_attn_fwd_packed (compact weights)
+static int attn_entry(const dash_problem* p, const void* Q, const void* K, const void* V,
+                      const float* w, const uint32_t* mask, void* O, float* lse, bool packed,
+                      void* stream) {
   int rc = check_problem(p, false);
   if (rc) return rc;
   if (!Q || !K || !V || !w || !mask || !O) return DASH_ERR_INVALID_ARG;
@@ -324,10 +347,12 @@ int dash_attn_fwd(const dash_problem* p, const void* Q, const void* K, const voi
         p->head_dim == 128
             ? dash::launch_attn_f32<128>(static_cast<const float*>(Q), static_cast<const float*>(K),
                                          static_cast<const float*>(V), w, mask, static_cast<float*>(O), lse,
-                                         p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, p->chunk, p->sigma, st)
+                                         p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, p->chunk, p->sigma,
+                                         st, packed)
             : dash::launch_attn_f32<64>(static_cast<const float*>(Q), static_cast<const float*>(K),
                                         static_cast<const float*>(V), w, mask, static_cast<float*>(O), lse,
-                                        p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, p->chunk, p->sigma, st);
+                                        p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, p->chunk, p->sigma,
+                                        st, packed);
     return cuda_status(e);
   }
   const int G = p->n_q_heads / p->n_kv_heads;
@@ -336,10 +361,26 @@ int dash_attn_fwd(const dash_problem* p, const void* Q, const void* K, const voi
   if (2 * (128 / G) > p->chunk || p->chunk % (2 * (128 / G)) != 0) return DASH_ERR_UNSUPPORTED;
   if (n_chunks(p) > 2048) return DASH_ERR_UNSUPPORTED;
   if (p->chunk == 64)
-    return p->head_dim == 128 ? run_attn_tc<64, 128>(p, Q, K, V, w, mask, O, lse, st)
-                              : run_attn_tc<64, 64>(p, Q, K, V, w, mask, O, lse, st);
-  return p->head_dim == 128 ? run_attn_tc<128, 128>(p, Q, K, V, w, mask, O, lse, st)
-                            : run_attn_tc<128, 64>(p, Q, K, V, w, mask, O, lse, st);
+    return p->head_dim == 128 ? run_attn_tc<64, 128>(p, Q, K, V, w, mask, O, lse, packed, st)
+                              : run_attn_tc<64, 64>(p, Q, K, V, w, mask, O, lse, packed, st);
+  return p->head_dim == 128 ? run_attn_tc<128, 128>(p, Q, K, V, w, mask, O, lse, packed, st)
+                            : run_attn_tc<128, 64>(p, Q, K, V, w, mask, O, lse, packed, st);
+}
+
+extern "C" {
+
+int dash_attn_fwd(const dash_problem* p, const void* Q, const void* K, const void* V,
+                  const float* w, const uint32_t* mask, void* O, float* lse, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  return attn_entry(p, Q, K, V, w, mask, O, lse, false, stream);
+}
+
+int dash_attn_fwd_packed(const dash_problem* p, const void* Q, const void* K, const void* V,
+                         const float* weight, const uint32_t* mask, void* O, float* lse,
+                         void* stream) {
+  return attn_entry(p, Q, K, V, weight, mask, O, lse, true, stream);
 }
 
 // dash_decode, dash_decode_varlen (lens: nullable device [batch]) and

@@ -211,8 +211,8 @@ template <typename T, int D, int NV, int KIND>
 __global__ void __launch_bounds__(256) route_kernel(
     const T* __restrict__ Q, const T* __restrict__ Kbar, float* __restrict__ w,
     uint32_t* __restrict__ mask, const T* __restrict__ K, const float* __restrict__ qbar,
-    int n_q, int n_kv, int seq, int chunk, int n_c, int kbar_rows, float xscale, float e,
-    int n_bg) {
+    int32_t* __restrict__ count, int32_t* __restrict__ index, int packed, int n_q, int n_kv,
+    int seq, int chunk, int n_c, int kbar_rows, float xscale, float e, int n_bg) {
   extern __shared__ __align__(16) float Ls[];
   __shared__ float khat[8][D];                 // estimate_diagonal: summary per position
   const int G = n_q / n_kv;
@@ -274,14 +274,33 @@ __global__ void __launch_bounds__(256) route_kernel(
   const float invG = 1.f / (float)G;
   const size_t row = ((size_t)bg * seq + pos0 + warp);
   float* wr = w + row * n_c;
+  const int nw = (n_c + 31) >> 5;
+  uint32_t* mr = mask + row * nw;
+  if (packed) {
+    // compact form: the routed chunks of the row in increasing order
+    int base = 0;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int c = lane + 32 * k;
+      const bool act = c < n_c && c < c_i && wacc[k] > 0.f;
+      const unsigned bits = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const int at = base + __popc(bits & ((1u << lane) - 1u));
+        wr[at] = wacc[k] * invG;
+        if (index) index[row * n_c + at] = c;
+      }
+      if (k < nw && lane == 0) mr[k] = bits;
+      base += __popc(bits);
+    }
+    if (count && lane == 0) count[row] = base;
+    return;
+  }
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
     const int c = lane + 32 * k;
     // a row of the first chunk with the diagonal candidate: weight 1 on it
     if (c < n_c) wr[c] = diag && n_elig == 0 ? (c == c_i ? 1.f : 0.f) : wacc[k] * invG;
   }
-  const int nw = (n_c + 31) >> 5;
-  uint32_t* mr = mask + row * nw;
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
     const int c = lane + 32 * k;
@@ -292,8 +311,9 @@ __global__ void __launch_bounds__(256) route_kernel(
 
 template <typename T, int D, int NV, int KIND>
 cudaError_t launch_route_nv(const T* Q, const T* Kbar, float* w, uint32_t* mask, const T* K,
-                            const float* qbar, int batch, int n_q, int n_kv, int seq, int chunk,
-                            float xscale, float e, cudaStream_t st) {
+                            const float* qbar, int32_t* count, int32_t* index, int packed,
+                            int batch, int n_q, int n_kv, int seq, int chunk, float xscale,
+                            float e, cudaStream_t st) {
   const int n_c = (seq + chunk - 1) / chunk;
   const int LS = ((n_c + 7) & ~7) + 4;
   const size_t smem = (size_t)16 * LS * sizeof(float);
@@ -302,19 +322,20 @@ cudaError_t launch_route_nv(const T* Q, const T* Kbar, float* w, uint32_t* mask,
   if (err != cudaSuccess) return err;
   const int n_bg = batch * n_kv;
   const unsigned grid = (unsigned)(n_bg * (seq / 8));
-  kern<<<grid, 256, smem, st>>>(Q, Kbar, w, mask, K, qbar, n_q, n_kv, seq, chunk, n_c, seq / chunk,
-                                xscale, e, n_bg);
+  kern<<<grid, 256, smem, st>>>(Q, Kbar, w, mask, K, qbar, count, index, packed, n_q, n_kv, seq,
+                                chunk, n_c, seq / chunk, xscale, e, n_bg);
   return cudaGetLastError();
 }
 
 template <typename T, int D, int KIND>
 cudaError_t launch_route_kind(const T* Q, const T* Kbar, float* w, uint32_t* mask, const T* K,
-                              const float* qbar, int batch, int n_q, int n_kv, int seq, int chunk,
-                              float xscale, float e, cudaStream_t st) {
+                              const float* qbar, int32_t* count, int32_t* index, int packed,
+                              int batch, int n_q, int n_kv, int seq, int chunk, float xscale,
+                              float e, cudaStream_t st) {
   const int n_c = (seq + chunk - 1) / chunk;
-#define DASH_RNV(NV)                                                                              \
-  launch_route_nv<T, D, NV, KIND>(Q, Kbar, w, mask, K, qbar, batch, n_q, n_kv, seq, chunk, xscale, \
-                                  e, st)
+#define DASH_RNV(NV)                                                                            \
+  launch_route_nv<T, D, NV, KIND>(Q, Kbar, w, mask, K, qbar, count, index, packed, batch, n_q,   \
+                                  n_kv, seq, chunk, xscale, e, st)
   if (n_c <= 128) return DASH_RNV(4);
   if (n_c <= 256) return DASH_RNV(8);
   if (n_c <= 512) return DASH_RNV(16);
@@ -324,21 +345,24 @@ cudaError_t launch_route_kind(const T* Q, const T* Kbar, float* w, uint32_t* mas
 }
 
 // K, qbar: non-null for estimate_diagonal (the keys and learned queries of
-// stage 0), else both null
+// stage 0), else both null.  packed: w is the compact form (count, index
+// nullable), else dense.
 template <typename T, int D>
 cudaError_t launch_route(const T* Q, const T* Kbar, float* w, uint32_t* mask, const T* K,
                          const float* qbar, int batch, int n_q, int n_kv, int seq, int chunk,
-                         float alpha, float gamma, cudaStream_t st) {
+                         float alpha, float gamma, cudaStream_t st, bool packed = false,
+                         int32_t* count = nullptr, int32_t* index = nullptr) {
   const float xscale = (alpha - 1.f) * gamma;
   const float e = 1.f / (alpha - 1.f);
+  const int pk = packed ? 1 : 0;
   if (alpha == 1.5f)
-    return launch_route_kind<T, D, kEntmax15>(Q, Kbar, w, mask, K, qbar, batch, n_q, n_kv, seq,
-                                               chunk, xscale, e, st);
+    return launch_route_kind<T, D, kEntmax15>(Q, Kbar, w, mask, K, qbar, count, index, pk, batch,
+                                               n_q, n_kv, seq, chunk, xscale, e, st);
   if (alpha == 2.f)
-    return launch_route_kind<T, D, kSparsemax>(Q, Kbar, w, mask, K, qbar, batch, n_q, n_kv, seq,
-                                                chunk, xscale, e, st);
-  return launch_route_kind<T, D, kEntmaxGeneric>(Q, Kbar, w, mask, K, qbar, batch, n_q, n_kv, seq,
-                                                  chunk, xscale, e, st);
+    return launch_route_kind<T, D, kSparsemax>(Q, Kbar, w, mask, K, qbar, count, index, pk, batch,
+                                                n_q, n_kv, seq, chunk, xscale, e, st);
+  return launch_route_kind<T, D, kEntmaxGeneric>(Q, Kbar, w, mask, K, qbar, count, index, pk,
+                                                  batch, n_q, n_kv, seq, chunk, xscale, e, st);
 }
 
 }  // namespace dash

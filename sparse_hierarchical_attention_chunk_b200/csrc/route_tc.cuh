@@ -49,6 +49,13 @@ struct RouteTcParams {
   const __nv_bfloat16* K;
   const float* qbar;
   int diag;
+  // compact form (packed != 0): w holds, per row, the weights of the routed
+  // chunks in increasing chunk order (entry k = the k-th set bit of the
+  // row's mask); index (nullable) their chunk numbers, count (nullable) how
+  // many there are
+  int packed;
+  int32_t* count;
+  int32_t* index;
   int n_q, n_kv, seq, chunk, n_c, nw, kbar_rows, n_tiles, n_bg, pos_base;
   float xscale, e;
 };
@@ -83,6 +90,11 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
   uint8_t* sKt = smem + Q_BYTES;                // 2 tile slots
+  // compact form: once the logits are in TMEM the Kbar tiles are free and
+  // hold the rows' weights and mask words until they are compacted
+  constexpr int NCMAX = SPLIT ? 1024 : 512;
+  float* wst = reinterpret_cast<float*>(sKt);                          // [NPOS][NCMAX]
+  uint32_t* mst = reinterpret_cast<uint32_t*>(sKt + NPOS * NCMAX * 4); // [NPOS][32]
 
   __shared__ __align__(8) uint64_t bar_q, bar_full[2], bar_empty[2], bar_logits;
   __shared__ uint32_t tmem_slot;
@@ -428,16 +440,24 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
           const int c = c0 + 2 * h;
           const float w0 = v[0] * invG, w1 = v[1] * invG;
           if (c0 < prm.n_c) {
-            // two scalar stores: with an odd n_c the row start is only 4-byte
-            // aligned (the half-warp still writes one contiguous 128-byte span)
-            if (c < prm.n_c) wrow[c] = w0;
-            if (c + 1 < prm.n_c) wrow[c + 1] = w1;
             // the query's own chunk (estimate_diagonal) is never a mask bit
             uint32_t bits = ((w0 > 0.f && c != c_i ? 1u : 0u) | (w1 > 0.f && c + 1 != c_i ? 2u : 0u))
                             << (2 * h);
 #pragma unroll
             for (int sh = 1; sh < 16; sh <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, sh);
-            if (h == 0) mrow[c0 >> 5] = bits;
+            if (prm.packed) {
+              // staged in shared memory; compacted once the row is complete
+              wst[pl * NCMAX + c] = w0;
+              wst[pl * NCMAX + c + 1] = w1;
+              if (h == 0) mst[pl * 32 + (c0 >> 5)] = bits;
+            } else {
+              // two scalar stores: with an odd n_c the row start is only
+              // 4-byte aligned (the half-warp still writes one contiguous
+              // 128-byte span)
+              if (c < prm.n_c) wrow[c] = w0;
+              if (c + 1 < prm.n_c) wrow[c + 1] = w1;
+              if (h == 0) mrow[c0 >> 5] = bits;
+            }
           }
         }
         return cnt;
@@ -453,14 +473,42 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
         if (redo) write_pass(bad || !cand ? tau : tc, false);
       }
       blocks_written = nblk;
+      if (prm.packed) {
+        // compact form: warp p writes position p's routed chunks in order
+        // (rank = set bits before them), its mask words and count
+        rows_sync();
+        if (warp < NPOS) {
+          const size_t rix = (size_t)bg * prm.seq + pos0 + warp;
+          float* wq = prm.w + rix * prm.n_c;
+          int32_t* iq = prm.index ? prm.index + rix * prm.n_c : nullptr;
+          uint32_t* mq = prm.mask + rix * prm.nw;
+          const int nwr = (n_elig + 31) >> 5;            // words holding routed chunks
+          int base = 0;
+          for (int k = 0; k < prm.nw; ++k) {
+            uint32_t bits = k < nwr ? mst[warp * 32 + k] : 0u;
+            if (k * 32 + 32 > n_elig) bits &= n_elig > k * 32 ? (1u << (n_elig - k * 32)) - 1u : 0u;
+            if ((bits >> lane) & 1u) {
+              const int at = base + __popc(bits & ((1u << lane) - 1u));
+              wq[at] = wst[warp * NCMAX + k * 32 + lane];
+              if (iq) iq[at] = k * 32 + lane;
+            }
+            if (lane == 0) mq[k] = bits;
+            base += __popc(bits);
+          }
+          if (lane == 0 && prm.count) prm.count[rix] = base;
+        }
+      }
     }
     // mask words / w columns not written above are 0: words
     // [c_base / 32 + blocks_written, nw) of this position's row (for SPLIT the
     // lower half covers all of words 0-15 whenever it has work)
-    const int zfirst = (c_base >> 5) + blocks_written;
+    const int zfirst = prm.packed ? (have ? prm.nw : 0) : (c_base >> 5) + blocks_written;
     const int zlast = SPLIT && !half ? min(16, prm.nw) : prm.nw;
+    if (prm.packed && !have && ch == 0 && (!SPLIT || !half) && (lane & 15) == 0 && prm.count)
+      prm.count[rowidx] = 0;                             // no eligible chunk: an empty row
     for (int k = zfirst + (lane & 15); ch == 0 && k < zlast; k += 16) {
       mrow[k] = 0u;
+      if (prm.packed) continue;
       for (int i = 0; i < 32 && k * 32 + i < prm.n_c; ++i) wrow[k * 32 + i] = 0.f;
       // estimate_diagonal on a row of the first chunk: the diagonal is the
       // only candidate, weight 1
@@ -514,11 +562,13 @@ cudaError_t launch_route_tc_part(const __nv_bfloat16* Q, const CUtensorMap& tk, 
   return launch_route_tc_k<SPLIT, kEntmaxGeneric>(tq, tk, prm, st);
 }
 
-// K, qbar: non-null for estimate_diagonal, else both null
+// K, qbar: non-null for estimate_diagonal, else both null.  packed: w is the
+// compact form (count, index nullable), else dense.
 inline cudaError_t launch_route_tc(const __nv_bfloat16* Q, const __nv_bfloat16* Kbar, float* w,
                                    uint32_t* mask, const __nv_bfloat16* K, const float* qbar,
                                    int batch, int n_q, int n_kv, int seq, int chunk, float alpha,
-                                   float gamma, cudaStream_t st) {
+                                   float gamma, cudaStream_t st, bool packed = false,
+                                   int32_t* count = nullptr, int32_t* index = nullptr) {
   const int n_c = (seq + chunk - 1) / chunk;
   CUtensorMap tk;
   {
@@ -533,6 +583,9 @@ inline cudaError_t launch_route_tc(const __nv_bfloat16* Q, const __nv_bfloat16* 
   prm.K = K;
   prm.qbar = qbar;
   prm.diag = K != nullptr;
+  prm.packed = packed ? 1 : 0;
+  prm.count = count;
+  prm.index = index;
   prm.n_q = n_q;
   prm.n_kv = n_kv;
   prm.seq = seq;

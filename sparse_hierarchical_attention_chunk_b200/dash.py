@@ -32,7 +32,7 @@ EXPORTED = ("dash_status_str", "dash_version", "dash_summarize", "dash_route", "
             "dash_workspace_bytes", "dash_decode", "dash_decode_varlen", "dash_decode_paged",
             "dash_get_error", "dash_decode_noalloc", "dash_summarize_append", "dash_route_topk",
             "dash_attn_bwd", "dash_route_bwd", "dash_summarize_bwd", "dash_selftest_wait_timeout",
-            "dash_selftest_exp2_poly")
+            "dash_selftest_exp2_poly", "dash_route_packed", "dash_attn_fwd_packed")
 
 
 class DashError(RuntimeError):
@@ -87,6 +87,10 @@ def lib():
         L.dash_attn_bwd.argtypes = [P] + [vp] * 13
         L.dash_route.restype = i32
         L.dash_route.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
+        L.dash_route_packed.restype = i32
+        L.dash_route_packed.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.dash_attn_fwd_packed.restype = i32
+        L.dash_attn_fwd_packed.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp]
         L.dash_attn_fwd.restype = i32
         L.dash_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.dash_workspace_bytes.restype = ctypes.c_size_t
@@ -290,6 +294,48 @@ def dash_route(p, Q, Kbar, w, mask, stream=None, K=None, qbar=None):
                                           _ptr(w), _ptr(mask), _stream(stream)))
 
 
+def dash_route_packed(p, Q, Kbar, mask, weight, count=None, index=None, stream=None, K=None,
+                      qbar=None):
+    """Stage 1 with compact weights: per row, the weights of the routed chunks
+    in increasing chunk order (weight), optionally their count and chunk
+    numbers (index).  Rows keep the dense row length n_c."""
+    dt = _tdtype(p)
+    rows = (p.batch, p.n_kv_heads, p.seq_len)
+    _check(Q, "Q", (p.batch, p.n_q_heads, p.seq_len, p.head_dim), dt)
+    _check(Kbar, "Kbar", (p.batch, p.n_kv_heads, p.seq_len // p.chunk, p.head_dim), dt)
+    _check(mask, "mask", rows + (n_words(p),), torch.int32)
+    _check(weight, "weight", rows + (n_chunks(p),), torch.float32)
+    if count is not None:
+        _check(count, "count", rows, torch.int32)
+    if index is not None:
+        _check(index, "index", rows + (n_chunks(p),), torch.int32)
+    if p.estimate_diagonal:
+        if K is None or qbar is None:
+            raise ValueError("estimate_diagonal needs K and qbar")
+        _check(K, "K", (p.batch, p.n_kv_heads, p.seq_len, p.head_dim), dt)
+        _check(qbar, "qbar", (p.n_kv_heads, p.head_dim), torch.float32)
+    _raise("dash_route_packed",
+           lib().dash_route_packed(ctypes.byref(p), _ptr(Q), _ptr(Kbar), _ptr(K), _ptr(qbar),
+                                   _ptr(mask), _ptr(count), _ptr(index), _ptr(weight),
+                                   _stream(stream)))
+
+
+def dash_attn_fwd_packed(p, Q, K, V, weight, mask, O, lse=None, stream=None):
+    """Stage 2 on the compact weights of dash_route_packed."""
+    dt = _tdtype(p)
+    _check(Q, "Q", (p.batch, p.n_q_heads, p.seq_len, p.head_dim), dt)
+    _check(K, "K", (p.batch, p.n_kv_heads, p.seq_len, p.head_dim), dt)
+    _check(V, "V", (p.batch, p.n_kv_heads, p.seq_len, p.head_dim), dt)
+    _check(weight, "weight", (p.batch, p.n_kv_heads, p.seq_len, n_chunks(p)), torch.float32)
+    _check(mask, "mask", (p.batch, p.n_kv_heads, p.seq_len, n_words(p)), torch.int32)
+    _check(O, "O", (p.batch, p.n_q_heads, p.seq_len, p.head_dim), dt)
+    if lse is not None:
+        _check(lse, "lse", (p.batch, p.n_q_heads, p.seq_len), torch.float32)
+    _raise("dash_attn_fwd_packed",
+           lib().dash_attn_fwd_packed(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(weight),
+                                      _ptr(mask), _ptr(O), _ptr(lse), _stream(stream)))
+
+
 def dash_workspace_bytes(p, is_decode):
     return int(lib().dash_workspace_bytes(ctypes.byref(p), 1 if is_decode else 0))
 
@@ -440,13 +486,19 @@ def alloc_prefill(p, device="cuda"):
     }
 
 
-def prefill(p, Q, K, V, qbar, out=None, stream=None, with_lse=True):
-    """Stage 0 -> stage 1 -> stage 2 on the device; returns the output dict."""
+def prefill(p, Q, K, V, qbar, out=None, stream=None, with_lse=True, packed=False):
+    """Stage 0 -> stage 1 -> stage 2 on the device; returns the output dict.
+    With packed, stage 1 writes the compact weights (out["w"] then holds, per
+    row, the routed chunks' weights in chunk order) and stage 2 reads them."""
     out = alloc_prefill(p, Q.device) if out is None else out
     dash_summarize(p, K, qbar, out["Kbar"], stream=stream)
+    lse = out["lse"] if with_lse else None
+    if packed:
+        dash_route_packed(p, Q, out["Kbar"], out["mask"], out["w"], stream=stream, K=K, qbar=qbar)
+        dash_attn_fwd_packed(p, Q, K, V, out["w"], out["mask"], out["O"], lse, stream=stream)
+        return out
     dash_route(p, Q, out["Kbar"], out["w"], out["mask"], stream=stream, K=K, qbar=qbar)
-    dash_attn_fwd(p, Q, K, V, out["w"], out["mask"], out["O"], out["lse"] if with_lse else None,
-                  stream=stream)
+    dash_attn_fwd(p, Q, K, V, out["w"], out["mask"], out["O"], lse, stream=stream)
     return out
 
 

@@ -255,6 +255,29 @@ def test_route_gqa_mean_and_shared_support():
     assert np.array_equal(m2, mask[:, :, pos])
 
 
+def test_pack_weights_against_the_dense_rows():
+    rng = np.random.default_rng(45)
+    B = 16
+    Q = rng.normal(size=(2, 4, 128, 8))
+    Kbar = rng.normal(size=(2, 2, 8, 8))
+    w, mask, _ = oracle.route(Q, Kbar, 1.5, 1.0, B)
+    count, index, weight = oracle.pack_weights(w, mask)
+    dense, m2 = oracle.unpack_weights(count, index, weight, 8)
+    np.testing.assert_array_equal(dense, w)
+    np.testing.assert_array_equal(m2, mask)
+    # a direct scan of each dense row, written out here
+    for b in range(2):
+        for g in range(2):
+            for i in range(128):
+                cs = [c for c in range(8) if w[b, g, i, c] > 0]
+                assert count[b, g, i] == len(cs) == bin(int(mask[b, g, i, 0])).count("1")
+                assert list(index[b, g, i, :len(cs)]) == cs
+                assert list(weight[b, g, i, :len(cs)]) == [w[b, g, i, c] for c in cs]
+                assert (index[b, g, i, len(cs):] == -1).all()
+    # rows of the first chunk are empty
+    assert not count[:, :, :B].any()
+
+
 # ----------------------------------------------------------------------------
 # estimate_diagonal: the query's own chunk as one more entmax candidate
 # ----------------------------------------------------------------------------

@@ -190,6 +190,103 @@ def test_route_tiny_f32():
 
 
 # ----------------------------------------------------------------------------
+# compact routing form: the routed chunks of each row and their weights
+# ----------------------------------------------------------------------------
+
+def _route_packed_case(wl, seed, diag=False):
+    inp = synth.make_prefill(wl, seed=seed)
+    kb = oracle_kbar(inp["K"], inp["qbar"], wl.chunk, _dt(wl)).cuda()
+    p = dash.problem_for(wl, estimate_diagonal=diag)
+    n_c, rows = wl.n_chunks, (wl.batch, wl.n_kv_heads, wl.seq)
+    Q, K, qb = inp["Q"].cuda(), inp["K"].cuda(), inp["qbar"].cuda()
+    w = torch.empty(rows + (n_c,), device="cuda")
+    mask = torch.empty(rows + ((n_c + 31) // 32,), dtype=torch.int32, device="cuda")
+    dash.dash_route(p, Q, kb, w, mask, K=K, qbar=qb)
+    pm = torch.empty_like(mask)
+    weight = torch.full(rows + (n_c,), 7.0, device="cuda")     # untouched past each count
+    index = torch.full(rows + (n_c,), -7, dtype=torch.int32, device="cuda")
+    count = torch.empty(rows, dtype=torch.int32, device="cuda")
+    dash.dash_route_packed(p, Q, kb, pm, weight, count, index, K=K, qbar=qb)
+    assert dash.dash_get_error() == dash.DASH_OK
+    return inp, kb, w, mask, pm, weight, index, count
+
+
+@pytest.mark.parametrize("name,diag", [("g16_d128_b64_nc37", False), ("g16_d128_b128_s05", False),
+                                       ("g8_d64_b64_batch2", False), ("alpha13_generic", False),
+                                       ("g16_d128_b64_nc37", True), ("g8_d64_b64_batch2", True)])
+def test_route_packed_is_the_dense_routing_compacted(name, diag):
+    wl = MED[name]
+    inp, kb, w, mask, pm, weight, index, count = _route_packed_case(wl, 38, diag)
+    # the same routing, written compactly: the same bits, and every listed
+    # weight is the dense kernel's weight at that chunk, in chunk order
+    assert torch.equal(pm, mask)
+    c_ref, i_ref, w_ref = oracle.pack_weights(np64(w), mask_from_dev(mask))
+    cnt = count.cpu().numpy()
+    assert (cnt == c_ref).all()
+    k = np.arange(wl.n_chunks)[None, None, None, :]
+    live = k < cnt[..., None]
+    assert (np.where(live, index.cpu().numpy(), -1) == i_ref).all()
+    assert (np.where(live, np64(weight), 0.0) == w_ref).all()
+    assert (np.where(live, 0, index.cpu().numpy() + 7) == 0).all()       # untouched past count
+    assert (np.where(live, 7.0, np64(weight)) == 7.0).all()
+    # and against the oracle's routing, packed
+    wr, mr, near = oracle.route(inp["Q"], kb.cpu(), wl.alpha, wl.gamma, wl.chunk,
+                                diag=(inp["K"], inp["qbar"]) if diag else None)
+    n_diff, n_bad = compare_masks(mask_from_dev(pm), mr, near, wl.n_chunks)
+    assert n_bad == 0
+    dense, _ = oracle.unpack_weights(cnt, index.cpu().numpy(), np64(weight), wl.n_chunks)
+    wr_routed = np.where(oracle.unpack_mask(mr, wl.n_chunks), wr, 0.0)
+    assert np.abs(dense - wr_routed).max() <= TOL_W
+
+
+def test_route_packed_more_than_512_chunks():
+    wl = W("med_split", "prefill", 1, 32, 2, 600 * 64, 128, 64, rho=(0.9, 0.2), needles=(3, 1))
+    inp, kb, w, mask, pm, weight, index, count = _route_packed_case(wl, 39)
+    assert torch.equal(pm, mask)
+    pos = np.array([0, 64, 511 * 64 + 5, 512 * 64, 530 * 64 + 63, 600 * 64 - 1])
+    c_ref, i_ref, w_ref = oracle.pack_weights(np64(w[:, :, pos]), mask_from_dev(mask[:, :, pos]))
+    cnt = count[:, :, pos].cpu().numpy()
+    assert (cnt == c_ref).all()
+    live = np.arange(wl.n_chunks)[None, None, None, :] < cnt[..., None]
+    assert (np.where(live, index[:, :, pos].cpu().numpy(), -1) == i_ref).all()
+    assert (np.where(live, np64(weight[:, :, pos]), 0.0) == w_ref).all()
+
+
+@pytest.mark.parametrize("name", ["g16_d128_b64_nc37", "g16_d128_b128_s05", "g4_d128_sigma0"])
+def test_attn_packed_gives_the_dense_bits(name):
+    wl = MED[name]
+    inp, kb, w, mask, pm, weight, index, count = _route_packed_case(wl, 40)
+    p = dash.problem_for(wl)
+    Q, K, V = inp["Q"].cuda(), inp["K"].cuda(), inp["V"].cuda()
+    O1, O2 = torch.empty_like(Q), torch.empty_like(Q)
+    l1 = torch.empty(Q.shape[:3], device="cuda")
+    l2 = torch.empty_like(l1)
+    dash.dash_attn_fwd(p, Q, K, V, w, mask, O1, l1)
+    dash.dash_attn_fwd_packed(p, Q, K, V, weight, pm, O2, l2)
+    assert dash.dash_get_error() == dash.DASH_OK
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+    Or, lr = oracle.attn_fwd(inp["Q"], inp["K"], inp["V"], np64(w), mask_from_dev(mask), wl.sigma,
+                             wl.chunk)
+    assert np.abs(np64(O2) - Or).max() <= TOL_O_BF16
+
+
+@pytest.mark.parametrize("zero_qbar", [False, True])
+def test_prefill_packed_tiny_f32(zero_qbar):
+    wl = configs.TINY_F32
+    inp = synth.make_prefill(wl, seed=41, zero_qbar=zero_qbar)
+    p = dash.problem_for(wl)
+    dev = [inp[n].cuda() for n in ("Q", "K", "V", "qbar")]
+    a = dash.prefill(p, *dev)
+    b = dash.prefill(p, *dev, packed=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a["mask"], b["mask"]) and torch.equal(a["O"], b["O"])
+    kb = oracle.chunk_summary(inp["K"], inp["qbar"], wl.chunk)
+    wr, mr, near = oracle.route(inp["Q"], kb, wl.alpha, wl.gamma, wl.chunk)
+    Or, _ = oracle.attn_fwd(inp["Q"], inp["K"], inp["V"], wr, mr, wl.sigma, wl.chunk)
+    assert np.abs(np64(b["O"]) - Or).max() <= TOL_O_F32
+
+
+# ----------------------------------------------------------------------------
 # stage 2
 # ----------------------------------------------------------------------------
 
