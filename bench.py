@@ -138,6 +138,22 @@ def prefill_work(wl, mask):
     return flops, exec_flops, frac.mean().item(), per_head
 
 
+def stage_bytes(wl, mask, packed=False):
+    """Algorithmic HBM bytes of stage 0 (K read, summaries written) and stage 1
+    (Q and summaries read, weights and mask written: the dense row of w, or
+    with the compact form only the routed entries)."""
+    b, hq, hkv, n, d, B = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.seq, wl.head_dim, wl.chunk
+    es = 2 if wl.dtype == "bf16" else 4
+    n_c = wl.n_chunks
+    kbar = b * hkv * (n // B) * d * es
+    s0 = b * hkv * n * d * es + kbar
+    nw = (n_c + 31) // 32
+    routed = popcount32(mask).sum().item()
+    w_bytes = routed * 4 if packed else b * hkv * n * n_c * 4
+    s1 = b * hq * n * d * es + kbar + w_bytes + b * hkv * n * nw * 4
+    return {"summarize": int(s0), "route": int(s1)}
+
+
 def decode_bytes(wl, mask, lens=None):
     """Algorithmic HBM bytes of one decode step (lens: per-sequence cache
     lengths, else wl.seq for all)."""
@@ -196,44 +212,68 @@ def run_ours(args, rank, world, device):
     def max_over_ranks(x):
         return shard.max_over_ranks(x, device)
 
-    def time_prefill(wl, steps, warmup, sigma=None, want_clocks=False):
+    def time_prefill(wl, steps, warmup, sigma=None, want_clocks=False, packed=False,
+                     keep_routing=False):
         inp = synth.make_prefill(wl, seed=rank, device=device)
         p = dash.problem_for(wl, sigma=sigma)
         Q, K, V, qbar = inp["Q"], inp["K"], inp["V"], inp["qbar"]
         out = dash.alloc_prefill(p, device)
         for _ in range(warmup):
-            dash.prefill(p, Q, K, V, qbar, out=out, with_lse=False)
+            dash.prefill(p, Q, K, V, qbar, out=out, with_lse=False, packed=packed)
         torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-                torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(steps)]
         barrier()
         torch.cuda.synchronize()
         sampler = ClockSampler(torch.cuda.current_device()) if want_clocks else None
         if sampler:
             sampler.__enter__()
-        for e0, ea, e1 in evs:
+        for e0, es, ea, e1 in evs:
             flush.fill_(1)
             e0.record(stream)
             dash.dash_summarize(p, K, qbar, out["Kbar"])
-            dash.dash_route(p, Q, out["Kbar"], out["w"], out["mask"])
+            es.record(stream)
+            if packed:
+                dash.dash_route_packed(p, Q, out["Kbar"], out["mask"], out["w"])
+            else:
+                dash.dash_route(p, Q, out["Kbar"], out["w"], out["mask"])
             ea.record(stream)
-            dash.dash_attn_fwd(p, Q, K, V, out["w"], out["mask"], out["O"])
+            if packed:
+                dash.dash_attn_fwd_packed(p, Q, K, V, out["w"], out["mask"], out["O"])
+            else:
+                dash.dash_attn_fwd(p, Q, K, V, out["w"], out["mask"], out["O"])
             e1.record(stream)
         torch.cuda.synchronize()
         if sampler:
             sampler.__exit__()
         barrier()
-        step_ms = [e0.elapsed_time(e1) for e0, ea, e1 in evs]
-        attn_ms = [ea.elapsed_time(e1) for e0, ea, e1 in evs]
+        step_ms = [e0.elapsed_time(e1) for e0, es, ea, e1 in evs]
+        sum_ms = [e0.elapsed_time(es) for e0, es, ea, e1 in evs]
+        route_ms = [es.elapsed_time(ea) for e0, es, ea, e1 in evs]
+        attn_ms = [ea.elapsed_time(e1) for e0, es, ea, e1 in evs]
         clocks = sampler.summary() if sampler else None
         flops, exec_flops, frac, per_head = prefill_work(wl, out["mask"])
         assert dash.dash_get_error() == dash.DASH_OK
         res = {"step_ms": max_over_ranks(statistics.mean(step_ms)),
                "attn_ms": max_over_ranks(statistics.mean(attn_ms)),
+               "sum_ms": max_over_ranks(statistics.mean(sum_ms)),
+               "route_ms": max_over_ranks(statistics.mean(route_ms)),
                "flops": flops, "exec_flops": exec_flops, "support": frac, "per_head": per_head,
-               "clocks": clocks, "inputs": (Q, K, V, qbar), "p": p}
+               "clocks": clocks, "inputs": (Q, K, V, qbar), "p": p,
+               "stage_bytes": stage_bytes(wl, out["mask"], packed)}
+        if keep_routing:
+            res["routing"] = {k: out[k].cpu() for k in ("Kbar", "w", "mask")}
         del out
         return res
+
+    def stage_rooflines(res):
+        """Achieved GB/s of stages 0 and 1 against the HBM peak."""
+        out = {}
+        for name, key in (("summarize", "sum_ms"), ("route", "route_ms")):
+            nb = res["stage_bytes"][name]
+            gbs = nb / (res[key] / 1e3) / 1e9
+            out[name] = {"ms": round(res[key], 4), "algorithmic_bytes": nb,
+                         "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        return out
 
     def time_topk_ablation(wl, steps, warmup):
         """Stage 2 on a fixed-budget top-k mask (the NSA / InfLLMv2-style
@@ -487,7 +527,7 @@ def run_ours(args, rank, world, device):
         if rank == 0:
             line["cpu_baseline"] = decode_cpu_baseline(wl, args.cpu_seconds)
         return line
-    main = time_prefill(wl, args.steps, args.warmup, want_clocks=True)
+    main = time_prefill(wl, args.steps, args.warmup, want_clocks=True, keep_routing=rank == 0)
     tokens_rank = wl.batch * wl.seq
     value = tokens_rank * world / (main["step_ms"] / 1e3)
     peak = peaks["bf16_tflops"]
@@ -500,7 +540,9 @@ def run_ours(args, rank, world, device):
                     "attn_fwd_tc", wl.name, "sparse_hierarchical_attention_chunk_b200/csrc/attn_tc.cuh"),
                 "algorithmic_flops_per_launch": main["flops"],
                 "tile_executed_flops_per_launch": main["exec_flops"],
+                "tile_executed_frac": round(main["exec_flops"] / (main["attn_ms"] / 1e3) / 1e12 / peak, 4),
                 "attn_ms": round(main["attn_ms"], 4)}
+    stages = stage_rooflines(main)
 
     # ------------------------------------------------------------- e2e: host buffers
     # Every step copies its inputs (Q, K, V, qbar) up from pinned host
@@ -568,22 +610,47 @@ def run_ours(args, rank, world, device):
         also.append(time_topk_ablation(wl, args.steps, args.warmup))
         # the stage-2 backward (reference kernel) on the 8k workload
         also.append(time_attn_bwd(configs.PREFILL_8K, min(args.steps, 5), args.warmup))
-        # 128k prefill (sigma sweep on the same inputs: time sigma = 1)
+        def prefill_entry(wlx, r, sigma=None, packed=False):
+            ax = r["flops"] / (r["attn_ms"] / 1e3) / 1e12
+            return {"workload": wlx.name, "metric": "prefill tokens/s",
+                    "sigma": wlx.sigma if sigma is None else sigma,
+                    "routing_form": "compact (dash_route_packed)" if packed else "dense w",
+                    "value": round(wlx.batch * wlx.seq * world / (r["step_ms"] / 1e3), 1),
+                    "ms_per_step": round(r["step_ms"], 3), "attn_ms": round(r["attn_ms"], 3),
+                    "roofline": {"bound": "tensor", "achieved": round(ax, 2), "peak": peak,
+                                 "unit": "TFLOP/s", "frac": round(ax / peak, 4),
+                                 "algorithmic_flops_per_launch": r["flops"],
+                                 "tile_executed_flops_per_launch": r["exec_flops"],
+                                 "tile_executed_frac": round(
+                                     r["exec_flops"] / (r["attn_ms"] / 1e3) / 1e12 / peak, 4),
+                                 "traffic": profile_traffic(
+                                     "attn_fwd_tc", wlx.name,
+                                     "sparse_hierarchical_attention_chunk_b200/csrc/attn_tc.cuh")
+                                 if sigma in (None, wlx.sigma) and not packed else None},
+                    "stages": stage_rooflines(r),
+                    "support_mean": round(r["support"], 4),
+                    "support_per_kv_head": [round(x, 4) for x in r["per_head"]]}
+
+        # 8k prefill
+        wl2 = configs.PREFILL_8K
+        r2 = time_prefill(wl2, args.steps, args.warmup)
+        also.append(prefill_entry(wl2, r2))
+        del r2
+        # the main workload with the compact routing form
+        rp = time_prefill(wl, args.steps, args.warmup, packed=True)
+        also.append(prefill_entry(wl, rp, packed=True))
+        del rp
+        torch.cuda.empty_cache()
+        # 128k prefill, sigma sweep on the same inputs (the support does not
+        # depend on sigma, only the prior's strength does)
         wl4 = configs.PREFILL_128K
-        r4 = time_prefill(wl4, max(2, min(args.steps, 3)), args.warmup)
-        a4 = r4["flops"] / (r4["attn_ms"] / 1e3) / 1e12
-        also.append({"workload": wl4.name, "metric": "prefill tokens/s",
-                     "value": round(wl4.batch * wl4.seq * world / (r4["step_ms"] / 1e3), 1),
-                     "ms_per_step": round(r4["step_ms"], 3), "attn_ms": round(r4["attn_ms"], 3),
-                     "roofline": {"bound": "tensor", "achieved": round(a4, 2), "peak": peak,
-                                  "unit": "TFLOP/s", "frac": round(a4 / peak, 4),
-                                  "algorithmic_flops_per_launch": r4["flops"],
-                                  "tile_executed_flops_per_launch": r4["exec_flops"],
-                                  "traffic": profile_traffic(
-                                      "attn_fwd_tc", wl4.name,
-                                      "sparse_hierarchical_attention_chunk_b200/csrc/attn_tc.cuh")},
-                     "support_mean": round(r4["support"], 4),
-                     "support_per_kv_head": [round(x, 4) for x in r4["per_head"]]})
+        for sg in (wl4.sigmas or (wl4.sigma,)):
+            r4 = time_prefill(wl4, max(2, min(args.steps, 3)), args.warmup, sigma=sg)
+            also.append(prefill_entry(wl4, r4, sigma=sg))
+            del r4
+            torch.cuda.empty_cache()
+        r4 = time_prefill(wl4, max(2, min(args.steps, 3)), args.warmup, packed=True)
+        also.append(prefill_entry(wl4, r4, packed=True))
         del r4
         torch.cuda.empty_cache()
         # decode, 8 sequences x 131072-token cache
@@ -606,13 +673,14 @@ def run_ours(args, rank, world, device):
                    "support_per_kv_head": [round(x, 4) for x in main["per_head"]],
                    "l2": "flushed (256 MiB write) before every timed step"},
         "roofline": roofline,
+        "stages": stages,
         "e2e": e2e,
         "gpu_launches": 3 * args.steps,
         "clocks": main["clocks"],
         "also": also,
     }
     if rank == 0:
-        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, main.get("routing"))
     return line
 
 
@@ -653,18 +721,45 @@ def oracle_sample_rate(wl, seconds, state, seed=0):
     return wl.batch * wl.seq / total, done, t_stage0 + t_rows
 
 
-def cpu_baseline(wl, seconds):
+def routing_flips(wl, state, routing, n_pos=64, seed=7):
+    """Mask bits of the timed run's routing that differ from the oracle's,
+    on a seeded sample of positions: stage 1 of the oracle on the GPU's own
+    summaries, compared bit by bit; flips are allowed only where some head's
+    score lies within 1e-4 of its threshold."""
+    import numpy as np
+    import oracle
+
+    inp = state[0]
+    rng = np.random.default_rng(seed)
+    pos = np.sort(rng.choice(np.arange(wl.chunk, wl.seq), size=n_pos, replace=False))
+    w, m, near = oracle.route(inp["Q"], routing["Kbar"], wl.alpha, wl.gamma, wl.chunk,
+                              positions=pos, near_tol=1e-4)
+    gm = routing["mask"].numpy().view(np.uint32)[:, :, pos]
+    a, b_ = oracle.unpack_mask(gm, wl.n_chunks), oracle.unpack_mask(m, wl.n_chunks)
+    diff = a != b_
+    wmax = float(np.abs(routing["w"].numpy()[:, :, pos].astype(np.float64) - w).max())
+    return {"positions": int(pos.size), "rows": int(pos.size * wl.batch * wl.n_kv_heads),
+            "mask_flips": int(diff.sum()), "flips_within_1e-4_of_tau": int((diff & near).sum()),
+            "flips_elsewhere": int((diff & ~near).sum()), "w_max_abs_err": wmax,
+            "how": "oracle stage 1 on the GPU's summaries at seeded positions (not timed)"}
+
+
+def cpu_baseline(wl, seconds, routing=None):
     try:
         from threadpoolctl import threadpool_info
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         threads = os.cpu_count()
-    rate, done, spent = oracle_sample_rate(wl, seconds, oracle_inputs(wl))
-    return {"value": round(rate, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "host_cpus": os.cpu_count(),
-            "sample": f"stage 0 on all chunks + stages 1-2 for {done} sampled query positions "
-                      f"(all heads), {spent:.1f} s of CPU time, extrapolated linearly to "
-                      f"{wl.seq} positions"}
+    state = oracle_inputs(wl)
+    rate, done, spent = oracle_sample_rate(wl, seconds, state)
+    res = {"value": round(rate, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "host_cpus": os.cpu_count(), "extrapolated": True,
+           "sample": f"stage 0 on all chunks + stages 1-2 for {done} sampled query positions "
+                     f"(all heads), {spent:.1f} s of CPU time, extrapolated linearly to "
+                     f"{wl.seq} positions"}
+    if routing is not None:
+        res["routing_parity"] = routing_flips(wl, state, routing)
+    return res
 
 
 def decode_cpu_baseline(wl, seconds):
@@ -753,7 +848,8 @@ def run_reference(args, rank, world):
         threads = os.cpu_count()
     return {"impl": "reference", "metric": f"prefill tokens/s (stage 0+1+2) at seq {wl.seq}",
             "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": round(ms, 1), "extrapolated": True,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(wl, world),
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
