@@ -66,11 +66,14 @@ __device__ __forceinline__ void summarize_chunk_warp(const T* __restrict__ base,
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
       // every lane now holds the score of its own row; gather all RPW scores
+      // (rows past `chunk` -- a partial last group, when the rows are the
+      // visible part of a chunk -- take no part: score -inf)
       float s[RPW];
       float smax = -INFINITY;
 #pragma unroll
       for (int r = 0; r < RPW; ++r) {
-        s[r] = __shfl_sync(0xffffffffu, part, r * LPR);
+        const float sr = __shfl_sync(0xffffffffu, part, r * LPR);
+        s[r] = row0 + r < chunk ? sr : -INFINITY;
         smax = fmaxf(smax, s[r]);
       }
       const float m_new = fmaxf(m, smax);
@@ -78,7 +81,7 @@ __device__ __forceinline__ void summarize_chunk_warp(const T* __restrict__ base,
       float psum = 0.f;
 #pragma unroll
       for (int r = 0; r < RPW; ++r) psum += __expf(s[r] - m_new);
-      const float pown = __expf(part - m_new);
+      const float pown = __expf((row0 + grp < chunk ? part : -INFINITY) - m_new);
       l = l * corr + psum;
 #pragma unroll
       for (int e = 0; e < EPV; ++e) acc[e] = fmaf(pown, x[e], acc[e] * corr);
