@@ -262,6 +262,7 @@ def run_ours(args, rank, world, device):
                "stage_bytes": stage_bytes(wl, out["mask"], packed)}
         if keep_routing:
             res["routing"] = {k: out[k].cpu() for k in ("Kbar", "w", "mask")}
+            res["routing"]["Q"] = Q.cpu()          # the very inputs the kernels read
         del out
         return res
 
@@ -721,7 +722,7 @@ def oracle_sample_rate(wl, seconds, state, seed=0):
     return wl.batch * wl.seq / total, done, t_stage0 + t_rows
 
 
-def routing_flips(wl, state, routing, n_pos=64, seed=7):
+def routing_flips(wl, routing, n_pos=64, seed=7):
     """Mask bits of the timed run's routing that differ from the oracle's,
     on a seeded sample of positions: stage 1 of the oracle on the GPU's own
     summaries, compared bit by bit; flips are allowed only where some head's
@@ -729,10 +730,9 @@ def routing_flips(wl, state, routing, n_pos=64, seed=7):
     import numpy as np
     import oracle
 
-    inp = state[0]
     rng = np.random.default_rng(seed)
     pos = np.sort(rng.choice(np.arange(wl.chunk, wl.seq), size=n_pos, replace=False))
-    w, m, near = oracle.route(inp["Q"], routing["Kbar"], wl.alpha, wl.gamma, wl.chunk,
+    w, m, near = oracle.route(routing["Q"], routing["Kbar"], wl.alpha, wl.gamma, wl.chunk,
                               positions=pos, near_tol=1e-4)
     gm = routing["mask"].numpy().view(np.uint32)[:, :, pos]
     a, b_ = oracle.unpack_mask(gm, wl.n_chunks), oracle.unpack_mask(m, wl.n_chunks)
@@ -758,7 +758,7 @@ def cpu_baseline(wl, seconds, routing=None):
                      f"(all heads), {spent:.1f} s of CPU time, extrapolated linearly to "
                      f"{wl.seq} positions"}
     if routing is not None:
-        res["routing_parity"] = routing_flips(wl, state, routing)
+        res["routing_parity"] = routing_flips(wl, routing)
     return res
 
 
