@@ -242,7 +242,7 @@ struct DecodeRouteParams {
 };
 
 template <int D, int KIND>
-__global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(256)
+__global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(256, 1)
 decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteParams prm) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
@@ -252,9 +252,13 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
   // boxes of CPC rows x 128 B)
   uint8_t* sKb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(route_smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t kb_bar;
-  __shared__ float X[2][kDecodeMaxChunks];    // logits of the (<= 2) heads this CTA owns
-  __shared__ float Pp[16][256];               // p of every head for this CTA's chunks
+  __shared__ __align__(8) uint64_t kb_bar[2];   // the two halves of the slice
+  // logits of every head for this CTA's chunks (read by the heads' owners
+  // after the first cluster barrier), then the staging of p of every head
+  // for this CTA's chunks (pulled from the heads' owners)
+  __shared__ __align__(16) float XP[16][256];
+  __shared__ __align__(16) float Pl[2][kDecodeMaxChunks];   // p of the (<= 2) heads this CTA owns
+  __shared__ float Xd[2];                     // estimate_diagonal: their diagonal logits
   __shared__ __align__(16) float red[2][2][4][4];   // float4 rows (Group4::sum4)
   __shared__ int cnt_all[kRouteCluster];
   __shared__ int wcnt[8];
@@ -285,19 +289,30 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int rows_here = max(0, min(CPC, c_q - c0));   // eligible chunks of this slice
   if (tid == 0) {
-    mbar_init(&kb_bar, 1);
+    mbar_init(&kb_bar[0], 1);
+    mbar_init(&kb_bar[1], 1);
     fence_mbar_init();
   }
   __syncthreads();
   if (tid == 0 && rows_here > 0) {
     tma_prefetch_desc(&tmKb);
-    mbar_arrive_expect_tx(&kb_bar, (uint32_t)((D / 64) * CPC * 128));
+    // two halves of CPC / 2 rows (a multiple of 16, so 1024-byte aligned in
+    // the swizzled tile): the first half's logits start while the second
+    // half is still in flight
+    // (the second half only when it holds eligible chunks: the warp whose
+    // first row of that half is eligible waits for it, so no copy is left
+    // in flight when the CTA exits)
 #pragma unroll
-    for (int kb = 0; kb < D / 64; ++kb)
-      tma_load_2d(sKb + kb * CPC * 128, &tmKb, &kb_bar, kb * 64, bg * prm.kbar_rows + c0);
+    for (int hf = 0; hf < (rows_here > CPC / 2 ? 2 : 1); ++hf) {
+      mbar_arrive_expect_tx(&kb_bar[hf], (uint32_t)((D / 64) * (CPC / 2) * 128));
+#pragma unroll
+      for (int kb = 0; kb < D / 64; ++kb)
+        tma_load_2d(sKb + kb * CPC * 128 + hf * (CPC / 2) * 128, &tmKb, &kb_bar[hf], kb * 64,
+                    bg * prm.kbar_rows + c0 + hf * (CPC / 2));
+    }
   }
 
-  // ---- logits of all heads for chunks [c0, c0 + CPC) -> owning CTAs
+  // ---- logits of all heads for chunks [c0, c0 + CPC), kept in this CTA
   {
     constexpr int KS = D / 16;
     const int gi = lane >> 2, t = lane & 3;
@@ -315,12 +330,16 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
       qa[kk][3] = v1 ? __ldg(q1 + kk * 8 + t + 4) : 0u;
     }
     // warp-uniform: the ldmatrix / mma below need the whole warp
-    const bool have = __all_sync(0xffffffffu, rows_here > 0 && mbar_wait(&kb_bar, 0, nullptr));
+    const bool have = __all_sync(0xffffffffu, rows_here > 0 && mbar_wait(&kb_bar[0], 0, nullptr));
     if (have) {
       const uint32_t sb = smem_u32(sKb);
+      bool second = false;                        // waited for the second half
       // pairs of n-tiles (16 chunks) per warp step; B fragments by ldmatrix
       for (int pr = warp; pr * 16 < rows_here; pr += 8) {
-        const int cb = c0 + pr * 16;
+        if (pr * 16 >= CPC / 2 && !second) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&kb_bar[1], 0, nullptr))) break;
+          second = true;
+        }
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         const int mi = lane >> 3, rr = lane & 7;
         const int row = pr * 16 + ((mi >> 1) << 3) + rr;
@@ -331,23 +350,22 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
           mma_bf16_16816(acc[0], qa[kk], b0, b1);
           mma_bf16_16816(acc[1], qa[kk], b2, b3);
         }
+        // chunks past c_q keep whatever the MMA gave: the owners read only
+        // the eligible ones
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int h = gi + (j >> 1) * 8;
-            const int c = cb + hf * 8 + 2 * t + (j & 1);
-            if (h < G && c < c_q) {
-              float* dst = cluster.map_shared_rank(&X[h % HPC][c], h / HPC);
-              *dst = acc[hf][j] * prm.xscale;
-            }
-          }
+        for (int hf = 0; hf < 2; ++hf) {
+          const int cl = pr * 16 + hf * 8 + 2 * t;
+          if (v0) *reinterpret_cast<float2*>(&XP[gi][cl]) =
+              make_float2(acc[hf][0] * prm.xscale, acc[hf][1] * prm.xscale);
+          if (v1) *reinterpret_cast<float2*>(&XP[gi + 8][cl]) =
+              make_float2(acc[hf][2] * prm.xscale, acc[hf][3] * prm.xscale);
+        }
       }
     }
   }
   // ---- estimate_diagonal: the query's own chunk c_q as one more candidate,
   // its logit against stage 0's summary of the cache rows c_q B .. L_b - 1,
-  // stored by the CTA that owns each head in X[slot][c_q]
+  // computed by the CTA that owns each head (Xd[slot])
   const bool dg = prm.diag != 0 && c_q > 0;
   if (dg && r * HPC < G) {                      // uniform over the CTA
     if (warp == 0) {
@@ -372,12 +390,15 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
       float acc = 0.f;
       for (int j = lane; j < D; j += 32) acc = fmaf(__bfloat162float(qh[j]), khat[j], acc);
       acc = warp_sum(acc);
-      if (lane == 0) X[warp][c_q] = acc * prm.xscale;
+      if (lane == 0) Xd[warp] = acc * prm.xscale;
     }
   }
   cluster.sync();
 
-  // ---- entmax of the owned heads, four warps per head -> p to the chunk owners
+  // ---- entmax of the owned heads, four warps per head.  Each thread pulls
+  // its 16 logits as four float4 (chunks 512 k + 4 tg .. + 3; a CTA's slice
+  // is a multiple of 32 chunks, so a float4 never straddles two CTAs) and
+  // keeps p in this CTA (Pl) for the chunk owners to pull.
   const int n_cand = c_q + (dg ? 1 : 0);        // candidates: eligible chunks (+ the diagonal)
   {
     const int slot = warp >> 2;
@@ -386,25 +407,60 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
       const int tg = tid & 127;
       float x[NV];
 #pragma unroll
-      for (int k = 0; k < NV; ++k) {
-        const int c = tg + 128 * k;
-        x[k] = c < n_cand ? X[slot][c] : -INFINITY;
+      for (int k = 0; k < NV / 4; ++k) {
+        const int c = 512 * k + 4 * tg;
+        float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        if (c < c_q) {
+          const int owner = c / CPC;
+          v = *cluster.map_shared_rank(reinterpret_cast<float4*>(&XP[h][c - owner * CPC]), owner);
+        }
+        x[4 * k + 0] = c + 0 < c_q ? v.x : (dg && c + 0 == c_q ? Xd[slot] : -INFINITY);
+        x[4 * k + 1] = c + 1 < c_q ? v.y : (dg && c + 1 == c_q ? Xd[slot] : -INFINITY);
+        x[4 * k + 2] = c + 2 < c_q ? v.z : (dg && c + 2 == c_q ? Xd[slot] : -INFINITY);
+        x[4 * k + 3] = c + 3 < c_q ? v.w : (dg && c + 3 == c_q ? Xd[slot] : -INFINITY);
       }
       Group4 gr{red[slot], warp & 3, lane, 1 + slot, 0};
       const float tau = entmax_tau_group<NV, KIND>(x, prm.e, gr);
 #pragma unroll
-      for (int k = 0; k < NV; ++k) {
-        const int c = tg + 128 * k;
+      for (int k = 0; k < NV / 4; ++k) {
+        const int c = 512 * k + 4 * tg;
         if (c < n_cand) {
-          const float pv = entmax_pow<KIND>(fmaxf(x[k] - tau, 0.f), prm.e);
-          const int owner = c / CPC;
-          float* dst = cluster.map_shared_rank(&Pp[h][c - owner * CPC], owner);
-          *dst = pv;
+          float4 pv;
+          pv.x = entmax_pow<KIND>(fmaxf(x[4 * k + 0] - tau, 0.f), prm.e);
+          pv.y = entmax_pow<KIND>(fmaxf(x[4 * k + 1] - tau, 0.f), prm.e);
+          pv.z = entmax_pow<KIND>(fmaxf(x[4 * k + 2] - tau, 0.f), prm.e);
+          pv.w = entmax_pow<KIND>(fmaxf(x[4 * k + 3] - tau, 0.f), prm.e);
+          *reinterpret_cast<float4*>(&Pl[slot][c]) = pv;
         }
       }
     }
   }
   cluster.sync();
+
+  // ---- p of every head for this CTA's chunks, pulled from the heads' owners
+  // (float4, in the order of the heads) into XP, whose logits are no longer
+  // read by anyone after the barrier above
+  {
+    // at most 16 heads x 64 float4 = 4 per thread: all four loads are in
+    // flight before any is stored
+    const int lim = min(CPC, n_cand - c0);      // this slice's candidate chunks
+    const int q4 = (lim + 3) >> 2;
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = tid + u * 256;
+      if (i < G * q4) {
+        const int hh = i / q4, cl = 4 * (i % q4);
+        v[u] = *cluster.map_shared_rank(reinterpret_cast<const float4*>(&Pl[hh % HPC][c0 + cl]), hh / HPC);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = tid + u * 256;
+      if (i < G * q4) *reinterpret_cast<float4*>(&XP[i / q4][4 * (i % q4)]) = v[u];
+    }
+  }
+  __syncthreads();
 
   // ---- GQA mean, mask words and this CTA's part of the active list
   const int c = c0 + tid;
@@ -413,7 +469,7 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
   if (tid < CPC && c < prm.n_c) {
     if (c < n_cand) {
       float s = 0.f;
-      for (int hh = 0; hh < G; ++hh) s += Pp[hh][tid];
+      for (int hh = 0; hh < G; ++hh) s += XP[hh][tid];
       wv = s / (float)G;
     } else if (prm.diag && c == c_q && c_q == 0) {
       wv = 1.f;                                   // the diagonal is the only candidate
@@ -618,6 +674,10 @@ __global__ void __launch_bounds__(160, 1) decode_split_kernel(
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // every K/V block is read once per step: keep it from evicting the
+      // partials and list the merge reads back (measured: ~8 us less per
+      // step on 8 x 128k caches)
+      const uint64_t pol = l2_evict_first_policy();
       int it = 0;
       for (; it < n_items; ++it) {
         const int s = it % NS;
@@ -627,8 +687,8 @@ __global__ void __launch_bounds__(160, 1) decode_split_kernel(
         mbar_arrive_expect_tx(&full[s], STAGE);
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb) {
-          tma_load_2d(st + kb * KV_BOX, &tmK, &full[s], kb * 64, row);
-          tma_load_2d(st + KV_BYTES + kb * KV_BOX, &tmV, &full[s], kb * 64, row);
+          tma_load_2d_hint(st + kb * KV_BOX, &tmK, &full[s], kb * 64, row, pol);
+          tma_load_2d_hint(st + KV_BYTES + kb * KV_BOX, &tmV, &full[s], kb * 64, row, pol);
         }
       }
       s_issued = it;
@@ -1065,7 +1125,7 @@ inline int run_decode(int batch, int n_q, int n_kv, int L, int D, int chunk, flo
     const uint64_t rows = (uint64_t)n_bg * (L / chunk);
     const uint64_t dims[2] = {(uint64_t)D, rows > 0 ? rows : 1};
     const uint64_t str[1] = {(uint64_t)D * 2};
-    const uint32_t box[2] = {64, (uint32_t)route_cpc(n_c)};
+    const uint32_t box[2] = {64, (uint32_t)route_cpc(n_c) / 2};   // half a slice
     if (!make_tmap(&tkb, rows > 0 ? Kbar : Kc, 2, dims, str, box)) return 3;
   }
   cudaError_t e = D == 128 ? launch_decode_route<128>(tkb, rp, n_bg, alpha, st)

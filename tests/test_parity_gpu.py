@@ -306,7 +306,7 @@ def _attn_case(wl, seed, sigma=None, dense=False, zero_qbar=False):
     lse = torch.empty(wl.batch, wl.n_q_heads, wl.seq, device="cuda")
     dash.dash_attn_fwd(p, inp["Q"].cuda(), inp["K"].cuda(), inp["V"].cuda(), to_dev(wr, torch.float32),
                        mask_to_dev(mr), O, lse)
-    torch.cuda.synchronize()
+    assert dash.dash_get_error() == dash.DASH_OK
     Or, lr = oracle.attn_fwd(inp["Q"], inp["K"], inp["V"], wr, mr, sigma, wl.chunk)
     return np64(O), np64(lse), Or, lr, inp
 
@@ -374,7 +374,7 @@ def test_end_to_end_bf16():
     inp = synth.make_prefill(wl, seed=11)
     p = dash.problem_for(wl)
     out = dash.prefill(p, inp["Q"].cuda(), inp["K"].cuda(), inp["V"].cuda(), inp["qbar"].cuda())
-    torch.cuda.synchronize()
+    assert dash.dash_get_error() == dash.DASH_OK
     ref_kb = oracle.chunk_summary(inp["K"], inp["qbar"], wl.chunk)
     kb = np64(out["Kbar"])
     assert np.all(np.abs(kb - ref_kb) <= 2.0 ** -8 * np.abs(ref_kb) + 1e-6)
@@ -451,6 +451,7 @@ def test_full_size_sampled_rows(wl):
         ps = dash.problem_for(wl, sigma=sg)
         O = torch.empty_like(dev["Q"])
         dash.dash_attn_fwd(ps, dev["Q"], dev["K"], dev["V"], w, mask, O)
+        assert dash.dash_get_error() == dash.DASH_OK
         Or, _ = oracle.attn_fwd(inp["Q"], inp["K"], inp["V"], np64(w)[:, :, pos],
                                 mask_from_dev(mask)[:, :, pos], sg, wl.chunk, positions=pos)
         assert np.abs(np64(O[:, :, pos]) - Or).max() <= TOL_O_BF16
