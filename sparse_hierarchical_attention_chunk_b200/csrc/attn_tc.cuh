@@ -112,17 +112,20 @@ __device__ __forceinline__ void exp2_poly2(uint64_t x, float& e0, float& e1) {
   e1 = __int_as_float(__float_as_int(t1) * 8388608 + __float_as_int(p1));
 }
 
-// Key blocks of BLK = 64 keys (a 128-key chunk is walked as two 64-key
-// sub-blocks sharing the chunk's routing bit and weight).
+// Key blocks of BLK keys, one chunk each (BLK = B = 64 or 128).
 template <int BLK, int D>
 struct TcLayout {
-  static_assert(BLK == 64, "64-key sub-blocks");
+  static_assert(BLK == 64 || BLK == 128, "64- or 128-key blocks");
   static constexpr int NT = 2;                      // tiles per CTA
-  static constexpr int NS = 3;                      // K and V ring depth
-  // Q is copied into TMEM and S = Q K^T runs as a TS-MMA, so the tensor core
-  // reads only K from shared memory (with Q from shared memory too, an
-  // N = 64 MMA needs more shared-memory bandwidth than there is).
-  static constexpr bool QTM = true;
+  static constexpr int NS = BLK == 64 ? 3 : 2;      // K and V ring depth
+  // With 64-key blocks Q is copied into TMEM and S = Q K^T runs as a
+  // TS-MMA, so the tensor core reads only K from shared memory (with Q from
+  // shared memory too, an N = 64 MMA needs more shared-memory bandwidth than
+  // there is).  With 128-key blocks S takes 128 TMEM columns per tile, which
+  // leaves no room for Q: S runs as an SS-MMA with N = 128 (half the
+  // shared-memory bytes per FLOP of N = 64), and each block step carries
+  // twice the MMA work for the same fixed per-step cost of the issuing warp.
+  static constexpr bool QTM = BLK == 64;
   static constexpr int QBOX = 128 * 128;            // 128 rows x 128 B (64 bf16 columns)
   static constexpr int Q_BYTES = QBOX * (D / 64);   // one tile
   static constexpr int KV_BOX = BLK * 128;          // BLK rows x 128 B
@@ -145,8 +148,8 @@ template <int CHUNK, int D>
 __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const AttnParams prm) {
-  constexpr int BLK = 64;                        // keys per MMA block
-  constexpr int SB = CHUNK / BLK;                // sub-blocks per chunk
+  constexpr int BLK = CHUNK;                     // keys per MMA block: one chunk
+  constexpr int SB = CHUNK / BLK;                // sub-blocks per chunk (1)
   using L = TcLayout<BLK, D>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -537,26 +540,38 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
 #pragma unroll
         for (int cc = 0; cc < BLK / 32; ++cc) tmem_st16u(tS + cc * 16, z);
       } else {
-        float sv[BLK];
-        tmem_ld64(tS, sv);
-        if (j == 0) {
-          const int lim = pos - (c * CHUNK + en.sb * BLK);   // causal: keys k <= lim are visible
+        // the block's S row in halves of 64 columns (one half for 64-key
+        // blocks, which stays in registers; two for 128-key blocks, read
+        // once for the max and once for the exponentials)
+        constexpr int NH = BLK / 64;
+        const int lim = j == 0 ? pos - (c * CHUNK + en.sb * BLK) : BLK;   // causal: keys k <= lim
+        float sv[64];
+        auto load_half = [&](int hh) {
+          tmem_ld64(tS + hh * 64, sv);
+          if (j == 0) {
 #pragma unroll
-          for (int k = 0; k < BLK; ++k) sv[k] = k <= lim ? sv[k] : -INFINITY;
+            for (int k = 0; k < 64; ++k) sv[k] = hh * 64 + k <= lim ? sv[k] : -INFINITY;
+          }
+        };
+        float mrow = -INFINITY;
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+          load_half(hh);
+          // row max: 8 independent partial maxima, three inputs per instruction
+          float mp[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mp[i] = sv[i];
+#pragma unroll
+          for (int k = 8; k < 64; k += 16)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mp[i] = fmax3(mp[i], sv[k + i], k + 8 + i < 64 ? sv[k + 8 + i] : sv[i]);
+#pragma unroll
+          for (int s2 = 4; s2 > 0; s2 >>= 1)
+#pragma unroll
+            for (int i = 0; i < s2; ++i) mp[i] = fmaxf(mp[i], mp[i + s2]);
+          mrow = fmaxf(mrow, mp[0]);
         }
-        // row max: 8 independent partial maxima, three inputs per instruction
-        float mp[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mp[i] = sv[i];
-#pragma unroll
-        for (int k = 8; k < BLK; k += 16)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mp[i] = fmax3(mp[i], sv[k + i], k + 8 + i < BLK ? sv[k + 8 + i] : sv[i]);
-#pragma unroll
-        for (int s2 = 4; s2 > 0; s2 >>= 1)
-#pragma unroll
-          for (int i = 0; i < s2; ++i) mp[i] = fmaxf(mp[i], mp[i + s2]);
-        const float mx = fmaf(mp[0], scale, bias);   // scale > 0: max commutes
+        const float mx = fmaf(mrow, scale, bias);   // scale > 0: max commutes
         // the first sub-block (diagonal, keys from the chunk start) always has a
         // visible key, so it sets a finite running max
         const float m_new = (jj == 0 || mx > m + 8.f) ? mx : m;
@@ -570,21 +585,38 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
         uint64_t rp[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) rp[i] = 0ull;
-        uint32_t pk[BLK / 2];
+        uint32_t pk[32];
+        // P of half hh as bf16 pairs, over S columns already read
+        auto store_p = [&](int hh) {
 #pragma unroll
-        for (int k2 = 0; k2 < BLK / 2; ++k2) {
-          const uint64_t x = f2_fma(f2_pack(sv[2 * k2], sv[2 * k2 + 1]), sc2, off2);
-          float e0, e1;
-          if (kPolyPairs & (1u << (k2 & 7))) {
-            exp2_poly2(x, e0, e1);
-          } else {
-            float x0, x1;
-            f2_unpack(x, x0, x1);
-            e0 = ex2f(x0);
-            e1 = ex2f(x1);
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = pk[cc * 16 + i];
+            tmem_st16u(tS + hh * 32 + cc * 16, v);
           }
-          rp[k2 & 3] = f2_add(rp[k2 & 3], f2_pack(e0, e1));
-          pk[k2] = pack_bf16x2(e0, e1);
+        };
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+          if (NH > 1) load_half(hh);
+#pragma unroll
+          for (int k2 = 0; k2 < 32; ++k2) {
+            const uint64_t x = f2_fma(f2_pack(sv[2 * k2], sv[2 * k2 + 1]), sc2, off2);
+            float e0, e1;
+            if (kPolyPairs & (1u << (k2 & 7))) {
+              exp2_poly2(x, e0, e1);
+            } else {
+              float x0, x1;
+              f2_unpack(x, x0, x1);
+              e0 = ex2f(x0);
+              e1 = ex2f(x1);
+            }
+            rp[k2 & 3] = f2_add(rp[k2 & 3], f2_pack(e0, e1));
+            pk[k2] = pack_bf16x2(e0, e1);
+          }
+          // a 128-key block writes its first half's P now (its S columns
+          // are read), a 64-key block after the rescale below
+          if (NH > 1) store_p(hh);
         }
         rp[0] = f2_add(f2_add(rp[0], rp[1]), f2_add(rp[2], rp[3]));
         float rs0, rs1;
@@ -616,13 +648,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
         }
         m = m_new;
         l += rs;
-#pragma unroll
-        for (int cc = 0; cc < BLK / 32; ++cc) {
-          uint32_t v[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = pk[cc * 16 + i];
-          tmem_st16u(tS + cc * 16, v);
-        }
+        if (NH == 1) store_p(0);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -660,20 +686,20 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
   }
 }
 
-template <int D>
+template <int BLK, int D>
 size_t attn_tc_smem_bytes(int n_c, int nw, int P) {
-  using L = TcLayout<64, D>;
+  using L = TcLayout<BLK, D>;
   return (size_t)L::OFF_AUX + (size_t)(n_c + 1) * 5 + 16 + (size_t)2 * P * nw * 8 +
          (size_t)L::NS * 2 * P * 4 + 1024;
 }
 
-// CHUNK = 64 or 128 (key blocks of 64), D = 64 or 128; K/V tensor maps use
-// {64, 64} boxes.
+// CHUNK = 64 or 128 (one key block per chunk), D = 64 or 128; K/V tensor
+// maps use {64, CHUNK} boxes.
 template <int CHUNK, int D>
 cudaError_t launch_attn_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                            const AttnParams& prm, cudaStream_t st) {
   auto kern = attn_fwd_tc_kernel<CHUNK, D>;
-  size_t smem = attn_tc_smem_bytes<D>(prm.n_c, prm.nw, prm.P);
+  size_t smem = attn_tc_smem_bytes<CHUNK, D>(prm.n_c, prm.nw, prm.P);
   // every CTA holds all 512 TMEM columns, so it must be alone on its SM:
   // ask for more than half of the shared memory
   if (smem < 118 * 1024) smem = 118 * 1024;

@@ -81,7 +81,7 @@ int run_attn_tc(const dash_problem* p, const void* Q, const void* K, const void*
   {
     const uint64_t dims[2] = {d, (uint64_t)p->batch * p->n_kv_heads * p->seq_len};
     const uint64_t str[1] = {d * 2};
-    const uint32_t box[2] = {64, 64};          // 64-key sub-blocks (two per 128-key chunk)
+    const uint32_t box[2] = {64, (uint32_t)CHUNK};   // one key block per chunk
     if (!make_tmap(&tk, K, 2, dims, str, box)) return DASH_ERR_CUDA;
     if (!make_tmap(&tv, V, 2, dims, str, box)) return DASH_ERR_CUDA;
   }
