@@ -210,23 +210,31 @@ int dash_attn_fwd(const dash_problem* p, const void* Q, const void* K, const voi
  * The pages state that the hierarchy is differentiable end to end
  * (gist.science summary, "Belangrijkste Bijdragen" item 1) but print no
  * gradients; these are the chain rule of stage 2's definition:
- * ds = p (dO.v - dO.O), dQ = ds K / sqrt(d), dK += ds^T Q / sqrt(d),
- * dV += p^T dO, and dw_c = sigma / w_c * (sum of ds over block c's keys and
+ * ds = p (dO.v - dO.O), dQ = ds K / sqrt(d), dK = ds^T Q / sqrt(d),
+ * dV = p^T dO, and dw_c = sigma / w_c * (sum of ds over block c's keys and
  * the KV group's heads) on every active routed block (the diagonal chunk's
  * bias is 0, the mask is piecewise constant: neither has a gradient).
  *   Q, K, V, w, mask, O, lse: the forward call's inputs and outputs (lse
  *   required); dO [b, Hq, N, d] (dtype of Q).
- *   dQ [b, Hq, N, d], dK, dV [b, Hkv, N, d] fp32: written (dK and dV are
- *   zeroed on the stream, then accumulated with atomics, so their summation
- *   order varies from run to run); dw [b, Hkv, N, n_c] fp32, nullable:
- *   written, 0 off the active routed blocks.
- * A reference kernel on CUDA cores (one warp per position and KV head), not
- * a tuned backward.  Errors: NULL or misaligned required pointers, a bad
- * problem -> DASH_ERR_INVALID_ARG; G > 16 -> DASH_ERR_UNSUPPORTED.
+ *   dQ [b, Hq, N, d], dK, dV [b, Hkv, N, d] fp32: written; dw
+ *   [b, Hkv, N, n_c] fp32, nullable: written, 0 off the active routed blocks.
+ *   workspace: dash_workspace_bytes(p, 2) bytes, 256-byte aligned (may be
+ *   NULL when that is 0).
+ * bf16 with d = 128 and G in {4, 8, 16} runs on tcgen05 tensor cores: a
+ * query-major kernel (dQ, dw; it also writes each row's dO.O and each
+ * 128-row tile's routed union to the workspace), then a key-major kernel
+ * (dK, dV) over the tiles that attend to each 128 keys; every output
+ * element is written once, in a fixed order (no atomics).  Other shapes run
+ * a reference kernel on CUDA cores that zeroes dK, dV on the stream and
+ * accumulates them with atomics (summation order varies from run to run).
+ * Errors: NULL or misaligned required pointers, a bad problem ->
+ * DASH_ERR_INVALID_ARG; G > 16 -> DASH_ERR_UNSUPPORTED; a missing, short or
+ * misaligned workspace -> DASH_ERR_WORKSPACE.
  */
 int dash_attn_bwd(const dash_problem* p, const void* Q, const void* K, const void* V,
                   const float* w, const uint32_t* mask, const void* O, const float* lse,
-                  const void* dO, float* dQ, float* dK, float* dV, float* dw, void* stream);
+                  const void* dO, float* dQ, float* dK, float* dV, float* dw, void* workspace,
+                  size_t workspace_bytes, void* stream);
 
 /*
  * Stage 1 backward: the gradient of dash_route's w for the cotangent dw,
@@ -268,8 +276,11 @@ int dash_attn_fwd_packed(const dash_problem* p, const void* Q, const void* K, co
                          const float* weight, const uint32_t* mask, void* O, float* lse,
                          void* stream);
 
-/* Workspace bytes needed by dash_attn_fwd (is_decode = 0) or dash_decode (1). */
-size_t dash_workspace_bytes(const dash_problem* p, int is_decode);
+/*
+ * Workspace bytes needed by dash_attn_fwd (which = 0), dash_decode and its
+ * variants (1) or dash_attn_bwd (2); 0 for an invalid problem or `which`.
+ */
+size_t dash_workspace_bytes(const dash_problem* p, int which);
 
 /*
  * Decode -- one new query per sequence at position L - 1 of an L-token cache

@@ -19,8 +19,11 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdash.so")
 
 SOURCES = ["dash.cu"]
-HEADERS = ["dash_common.cuh", "tmap.cuh", "tmem_wide.cuh", "summarize.cuh", "route.cuh", "route_tc.cuh", "route_topk.cuh", "attn_bwd.cuh", "route_bwd.cuh",
-           "attn_tc.cuh", "attn_f32.cuh", "decode.cuh"]
+
+
+def _headers():
+    """Every header of csrc/ (all are reachable from dash.cu)."""
+    return sorted(f for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -42,7 +45,7 @@ def _stale():
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "dash.h"),
+    deps = [os.path.join(CSRC, f) for f in SOURCES + _headers()] + [os.path.join(INCLUDE, "dash.h"),
                                                                   os.path.abspath(__file__)]
     return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
 

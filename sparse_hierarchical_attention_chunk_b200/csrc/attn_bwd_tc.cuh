@@ -1,0 +1,834 @@
+// Stage 2 backward on tcgen05 (bf16, G query heads per KV head, d = 128).
+//
+// The chain rule of the prior-induced block-sparse softmax of the
+// gist.science technical summary, "Fase 2" (the pages state end-to-end
+// differentiability, "Belangrijkste Bijdragen" item 1, and print no
+// gradients).  For a row (position i, query head h) and its active keys j,
+// s_j = q.k_j / sqrt(d) + beta_j, p = softmax(s) (recomputed from the
+// forward's log-normaliser), with the cotangent do and D = do.o:
+//   dp_j = do.v_j,  ds_j = p_j (dp_j - D),
+//   dq = sum_j ds_j k_j / sqrt(d),  dk_j = sum_rows ds_j q / sqrt(d),
+//   dv_j = sum_rows p_j do,  dw_c = sigma / w_c sum_{j in c, group heads} ds_j.
+// Two kernels, neither with atomics (every output element is written by one
+// CTA, in a fixed order):
+//
+//   attn_bwd_dq_kernel   query-major, like the forward: one tile of M = 128
+//       rows (P = 128 / G positions x G heads) per CTA walks the diagonal
+//       chunk and the union of its positions' routed chunks in 64-key blocks.
+//       Per block: S = Q K^T and dP = dO V^T (TS-MMAs, Q and dO copied into
+//       TMEM), then the softmax warps form P and dS (written as bf16 over S)
+//       and the row sums of dS (-> dw, summed over the heads of a position by
+//       shuffles), then dQ += dS K (K as the MN-major operand).  S/dP are
+//       double-buffered, so block n+1's S and dP run while block n's dS is
+//       formed.  Also writes D per row, for the key-major kernel.
+//   attn_bwd_dkv_kernel  key-major: one CTA per 128 keys (one 128-key chunk
+//       or a pair of 64-key chunks) walks the query tiles whose rows attend to
+//       those keys (the tiles of the keys' own chunks, causal, and every later
+//       tile one of whose positions routes to them, found from the mask).  Per
+//       tile: S^T = K Q^T and dP^T = V dO^T (SS-MMAs, M = 128 keys, N = 128
+//       rows), P^T and dS^T by the key threads (lse, D and the bias of each
+//       row broadcast from shared memory), then dV += P^T dO and
+//       dK += dS^T Q with the accumulators in TMEM for the whole walk.
+#pragma once
+
+#include <cuda.h>
+#include "dash_common.cuh"
+#include "tmem_wide.cuh"
+#include "attn_tc.cuh"
+
+namespace dash {
+
+struct BwdParams {
+  const float* w;
+  const uint32_t* mask;
+  const float* lse;
+  const __nv_bfloat16* O;
+  const __nv_bfloat16* dO;
+  float* dQ;
+  float* dK;
+  float* dV;
+  float* dw;             // nullable
+  float* Drow;           // [b, n_q, seq]: dO . O (written by the dQ kernel)
+  uint32_t* tmask;       // [b * n_kv, nw, n_tiles]: each tile's routed union (dQ kernel)
+  int n_q, n_kv, seq, chunk, n_c, nw, G, lgG, P, n_tiles, n_bg;
+  float sigma, scale_log2, scale;
+};
+
+// ---------------------------------------------------------------------------
+// dQ and dw
+// ---------------------------------------------------------------------------
+template <int CHUNK>
+__global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    const BwdParams prm) {
+  constexpr int D = 128;
+  constexpr int BLK = 64;                        // keys per block
+  constexpr int SB = CHUNK / BLK;                // sub-blocks per chunk
+  constexpr int NS = 3;                          // K / V ring depth
+  constexpr int QBOX = 128 * 128;                // 128 rows x 128 B
+  constexpr int T_BYTES = 2 * QBOX;              // one 128 x 128 bf16 tile
+  constexpr int KV_BOX = BLK * 128;
+  constexpr int KV_BYTES = 2 * KV_BOX;
+  // TMEM columns: Q | dO (bf16 pairs) | dQ (fp32) | S, dP of buffer 0 | of buffer 1
+  constexpr uint32_t TM_Q = 0, TM_DO = 64, TM_DQ = 128, TM_BUF = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sdO = sQ + T_BYTES;
+  uint8_t* sK = sdO + T_BYTES;
+  uint8_t* sV = sK + NS * KV_BYTES;
+  int* list = reinterpret_cast<int*>(sV + NS * KV_BYTES);                // [n_c + 1]
+  uint32_t* mrows = reinterpret_cast<uint32_t*>(list + prm.n_c + 1);     // [P][nw]
+  float* w_sm = reinterpret_cast<float*>(mrows + prm.P * prm.nw);        // [NS][P]
+
+  __shared__ __align__(8) uint64_t bar_qd, bar_qd_tm, bar_s_full[2], bar_ds_full[2], bar_fin;
+  __shared__ __align__(8) uint64_t bar_k_full[NS], bar_k_empty[NS], bar_v_full[NS], bar_v_empty[NS];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int nb_s;
+  __shared__ volatile int abort_s;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = prm.n_tiles - 1 - (int)(blockIdx.x % prm.n_tiles);   // late tiles first
+  const int bg = (int)(blockIdx.x / prm.n_tiles);
+  const int b = bg / prm.n_kv, g = bg % prm.n_kv;
+  const int P = prm.P, G = prm.G;
+  const int pos0 = tile * P;
+  const int c_i = pos0 / CHUNK;
+  const int n_wl = min(P, 32);
+
+  if (warp == 5) {
+    tmem_alloc(&tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_qd, 1);
+    mbar_init(&bar_qd_tm, 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar_s_full[t], 1);
+      mbar_init(&bar_ds_full[t], 128);
+    }
+    mbar_init(&bar_fin, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar_k_full[s], 1);
+      mbar_init(&bar_k_empty[s], 1);
+      mbar_init(&bar_v_full[s], 1 + n_wl);
+      mbar_init(&bar_v_empty[s], 1);
+    }
+    abort_s = 0;
+    fence_mbar_init();
+  }
+  const size_t row0 = (size_t)bg * prm.seq + pos0;
+  for (int i = tid; i < P * prm.nw; i += blockDim.x) mrows[i] = prm.mask[row0 * prm.nw + i];
+  __syncthreads();
+  // block list: the diagonal chunk, then the union of the routed chunks c < c_i
+  if (warp == 0) {
+    int base = 1;
+    for (int k0 = 0; k0 < prm.nw; k0 += 32) {
+      const int k = k0 + lane;
+      uint32_t u = 0;
+      if (k < prm.nw && k * 32 < c_i) {
+        for (int p = 0; p < P; ++p) u |= mrows[p * prm.nw + k];
+        const int rem = c_i - k * 32;
+        if (rem < 32) u &= (1u << rem) - 1u;
+      }
+      if (k < prm.nw) prm.tmask[((size_t)bg * prm.nw + k) * prm.n_tiles + tile] = u;
+      const int cnt = __popc(u);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int at = base + incl - cnt;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1;
+        list[at++] = k * 32 + bit;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      list[0] = c_i;
+      nb_s = base;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const int nb = nb_s;
+  // walk: the diagonal chunk's sub-blocks (the second only if a position
+  // reaches it), then SB sub-blocks per routed chunk
+  const int diag_lo = c_i * CHUNK;
+  const int n_diag = (SB == 2 && pos0 + P - 1 >= diag_lo + BLK) ? 2 : 1;
+  const int nbb = n_diag + (nb - 1) * SB;
+  struct Entry { int j, c, sb; };
+  auto entry = [&](int jj) {
+    Entry e;
+    if (jj < n_diag) {
+      e.j = 0; e.c = c_i; e.sb = jj;
+    } else {
+      const int r = jj - n_diag;
+      e.j = 1 + r / SB; e.sb = r % SB; e.c = list[e.j];
+    }
+    return e;
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar_qd, 2 * T_BYTES);
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb) {
+        tma_load_3d(sQ + kb * QBOX, &tmQ, &bar_qd, kb * 64, b * prm.n_q + g * G, pos0);
+        tma_load_3d(sdO + kb * QBOX, &tmdO, &bar_qd, kb * 64, b * prm.n_q + g * G, pos0);
+      }
+    }
+    int issued_k = 0, issued_v = 0;
+    for (int j = 0; j < nbb; ++j) {
+      const int s = j % NS;
+      const uint32_t par = ((j / NS) & 1) ^ 1;
+      const Entry en = entry(j);
+      const int krow = bg * prm.seq + en.c * CHUNK + en.sb * BLK;
+      int okw = lane == 0 ? (int)mbar_wait(&bar_k_empty[s], par, &abort_s) : 0;
+      if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar_k_full[s], KV_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_2d(sK + s * KV_BYTES + kb * KV_BOX, &tmK, &bar_k_full[s], kb * 64, krow);
+      }
+      issued_k = j + 1;
+      okw = lane == 0 ? (int)mbar_wait(&bar_v_empty[s], par, &abort_s) : 0;
+      if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar_v_full[s], KV_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_2d(sV + s * KV_BYTES + kb * KV_BOX, &tmV, &bar_v_full[s], kb * 64, krow);
+      }
+      if (lane < n_wl) {
+        for (int q = lane; q < P; q += 32)
+          cp_async_4(w_sm + s * P + q, prm.w + (row0 + q) * prm.n_c + en.c);
+        cp_async_arrive_noinc(&bar_v_full[s]);
+      }
+      issued_v = j + 1;
+    }
+    if (abort_s) {
+      if (lane == 0) {
+        for (int j = (issued_k > NS ? issued_k - NS : 0); j < issued_k; ++j)
+          mbar_wait(&bar_k_full[j % NS], (j / NS) & 1, nullptr);
+        for (int j = (issued_v > NS ? issued_v - NS : 0); j < issued_v; ++j)
+          mbar_wait(&bar_v_full[j % NS], (j / NS) & 1, nullptr);
+      }
+      cp_async_wait_all();
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    // S(n), dP(n) into buffer n & 1; after block n's dS: dQ(n), then S(n+2),
+    // dP(n+2) into the same buffer (in issue order, after dQ(n) read dS(n)).
+    constexpr uint32_t idS = idesc_bf16_f32(128, BLK, 0, 0);
+    constexpr uint32_t idQ = idesc_bf16_f32(128, D, 0, 1);
+    const bool leader = elect_one();
+    const uint64_t dK0 = sw128_desc(smem_u32(sK), 16, 1024);
+    const uint64_t dV0 = sw128_desc(smem_u32(sV), 16, 1024);
+    const uint64_t dKmn0 = sw128_desc(smem_u32(sK), KV_BOX, 1024);   // K as the MN-major operand
+    int n_s = 0, n_q = 0;
+    auto wait_all = [&](uint64_t* bar, uint32_t par) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, &abort_s));
+    };
+    auto issue_sdp = [&](int n) {            // S(n), dP(n); K(n), V(n) loaded
+      const int s = n % NS;
+      const uint32_t buf = tmem + TM_BUF + (uint32_t)(n & 1) * 128;
+      const uint64_t dk = dK0 + (uint64_t)((s * KV_BYTES) >> 4);
+      const uint64_t dv = dV0 + (uint64_t)((s * KV_BYTES) >> 4);
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t offk = (kk >> 2) * KV_BOX + (kk & 3) * 32;
+          tc_mma_ts(buf, tmem + TM_Q + kk * 8, dk + (offk >> 4), idS, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t offk = (kk >> 2) * KV_BOX + (kk & 3) * 32;
+          tc_mma_ts(buf + 64, tmem + TM_DO + kk * 8, dv + (offk >> 4), idS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bar_s_full[n & 1]);
+      }
+      __syncwarp();
+      ++n_s;
+    };
+    bool ok = wait_all(&bar_qd_tm, 0);
+    for (int n = 0; ok && n < 2 && n < nbb; ++n) {
+      if (!(ok = wait_all(&bar_k_full[n % NS], (n / NS) & 1) &&
+                 wait_all(&bar_v_full[n % NS], (n / NS) & 1)))
+        break;
+      tc_fence_after();
+      issue_sdp(n);
+    }
+    for (int n = 0; ok && n < nbb; ++n) {
+      const int s = n % NS;
+      if (!(ok = wait_all(&bar_ds_full[n & 1], (n >> 1) & 1))) break;
+      tc_fence_after();
+      const uint32_t ds = tmem + TM_BUF + (uint32_t)(n & 1) * 128;   // dS(n), bf16 pairs
+      const uint64_t dkm = dKmn0 + (uint64_t)((s * KV_BYTES) >> 4);
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < BLK / 16; ++kk)
+          tc_mma_ts(tmem + TM_DQ, ds + kk * 8, dkm + (uint64_t)((kk * 2048) >> 4), idQ,
+                    (n > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&bar_k_empty[s]);
+        tc_commit(&bar_v_empty[s]);
+        if (n + 1 == nbb) tc_commit(&bar_fin);
+      }
+      __syncwarp();
+      ++n_q;
+      if (n + 2 < nbb) {
+        const int s2 = (n + 2) % NS;
+        if (!(ok = wait_all(&bar_k_full[s2], ((n + 2) / NS) & 1) &&
+                   wait_all(&bar_v_full[s2], ((n + 2) / NS) & 1)))
+          break;
+        tc_fence_after();
+        issue_sdp(n + 2);
+      }
+    }
+    if (abort_s && lane == 0) {
+      if (n_s > 0) mbar_wait(&bar_s_full[(n_s - 1) & 1], ((n_s - 1) >> 1) & 1, nullptr);
+      if (n_q > 0) mbar_wait(&bar_k_empty[(n_q - 1) % NS], ((n_q - 1) / NS) & 1, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ rows (warps 0-3)
+    const int r = tid;                         // row = TMEM lane
+    const int p = r / G, hq = r % G;
+    const int pos = pos0 + p;
+    const int qh = g * G + hq;
+    const uint32_t tlane = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t* mrow = mrows + p * prm.nw;
+    const size_t qrow = ((size_t)b * prm.n_q + qh) * prm.seq + pos;
+    const float scale = prm.scale_log2, sigma = prm.sigma;
+    const float lse2 = prm.lse[qrow] * 1.4426950408889634f;
+    // D = dO . O of this row (fp32), also kept for the key-major kernel
+    float Dr = 0.f;
+    {
+      const uint4* orow = reinterpret_cast<const uint4*>(prm.O + qrow * D);
+      const uint4* drow = reinterpret_cast<const uint4*>(prm.dO + qrow * D);
+#pragma unroll 4
+      for (int v = 0; v < D / 8; ++v) {
+        const uint4 a = __ldg(orow + v), c = __ldg(drow + v);
+        const __nv_bfloat16* xa = reinterpret_cast<const __nv_bfloat16*>(&a);
+        const __nv_bfloat16* xc = reinterpret_cast<const __nv_bfloat16*>(&c);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) Dr = fmaf(__bfloat162float(xa[e]), __bfloat162float(xc[e]), Dr);
+      }
+      prm.Drow[qrow] = Dr;
+    }
+    // waits are made warp-uniform: the TMEM loads / stores and shuffles below
+    // are warp-collective
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_qd, 0, &abort_s));
+    // Q and dO rows: shared memory (TMA, 128-byte swizzle) -> TMEM as bf16 pairs
+    if (ok) {
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint8_t* base = (which ? sdO : sQ) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          uint32_t v[32];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 q4 = *reinterpret_cast<const uint4*>(base + kb * QBOX + ((ch ^ (r & 7)) << 4));
+            v[ch * 4 + 0] = q4.x;
+            v[ch * 4 + 1] = q4.y;
+            v[ch * 4 + 2] = q4.z;
+            v[ch * 4 + 3] = q4.w;
+          }
+          uint32_t h0[16], h1[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            h0[i] = v[i];
+            h1[i] = v[16 + i];
+          }
+          const uint32_t dst = tmem + tlane + (which ? TM_DO : TM_Q) + kb * 32;
+          tmem_st16u(dst, h0);
+          tmem_st16u(dst + 16, h1);
+        }
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(&bar_qd_tm);
+    float dsum_chunk = 0.f;                    // dS summed over a routed chunk's sub-blocks
+    for (int n = 0; ok && n < nbb; ++n) {
+      const Entry en = entry(n);
+      const int c = en.c;
+      const bool act = en.j == 0 || ((mrow[c >> 5] >> (c & 31)) & 1u);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_s_full[n & 1], (n >> 1) & 1, &abort_s))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float bias = 0.f;
+      float wc = 0.f;
+      if (en.j > 0) {
+        // the routing weights of block n (cp.async, counted on V's barrier)
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_v_full[n % NS], (n / NS) & 1, &abort_s))) {
+          ok = false;
+          break;
+        }
+        if (!act) {
+          bias = -INFINITY;
+        } else {
+          wc = w_sm[(n % NS) * P + p];
+          if (sigma != 0.f) bias = sigma * lg2f(wc);
+        }
+      }
+      const uint32_t tb = tmem + tlane + TM_BUF + (uint32_t)(n & 1) * 128;
+      float dsum = 0.f;
+      if (!__any_sync(0xffffffffu, act)) {
+        uint32_t z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0u;
+        tmem_st16u(tb, z);
+        tmem_st16u(tb + 16, z);
+      } else {
+        float sv[64], dp[64];
+        tmem_ld64(tb, sv);
+        tmem_ld64(tb + 64, dp);
+        const int lim = en.j == 0 ? pos - (c * CHUNK + en.sb * BLK) : BLK;   // causal on the diagonal
+        const float off = bias - lse2;
+        uint32_t pk[32];
+#pragma unroll
+        for (int k2 = 0; k2 < 32; ++k2) {
+          float d2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int k = 2 * k2 + u;
+            const float pr = k <= lim ? ex2f(fmaf(sv[k], scale, off)) : 0.f;
+            d2[u] = pr * (dp[k] - Dr);
+            dsum += d2[u];
+          }
+          pk[k2] = pack_bf16x2(d2[0], d2[1]);
+        }
+        uint32_t h0[16], h1[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          h0[i] = pk[i];
+          h1[i] = pk[16 + i];
+        }
+        tmem_st16u(tb, h0);
+        tmem_st16u(tb + 16, h1);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_ds_full[n & 1]);
+      // dw of a routed chunk: sigma / w times the sum of dS over its keys and
+      // the heads of the position (adjacent lanes), written once per chunk
+      if (en.j > 0 && prm.dw && sigma != 0.f) {
+        dsum_chunk += dsum;
+        if (en.sb == SB - 1) {
+          float tot = dsum_chunk;
+          for (int o = 1; o < G; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+          if (hq == 0 && act)
+            prm.dw[((size_t)bg * prm.seq + pos) * prm.n_c + c] = wc > 0.f ? sigma / wc * tot : 0.f;
+          dsum_chunk = 0.f;
+        }
+      }
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_fin, 0, &abort_s))) {
+      tc_fence_after();
+      float* drow = prm.dQ + qrow * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float o[32];
+        tmem_ld32(tmem + tlane + TM_DQ + cc * 32, o);
+        float4* dst = reinterpret_cast<float4*>(drow + cc * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          dst[q4] = make_float4(o[4 * q4] * prm.scale, o[4 * q4 + 1] * prm.scale,
+                                o[4 * q4 + 2] * prm.scale, o[4 * q4 + 3] * prm.scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+inline size_t attn_bwd_dq_smem_bytes(int n_c, int nw, int P) {
+  return (size_t)2 * 2 * 128 * 128 + (size_t)3 * 2 * 2 * 64 * 128 + (size_t)(n_c + 1) * 4 +
+         (size_t)P * nw * 4 + (size_t)3 * P * 4 + 1024 + 64;
+}
+
+// ---------------------------------------------------------------------------
+// dK and dV
+// ---------------------------------------------------------------------------
+// Per-tile row data staged beside the tile's Q and dO (head-major, as they
+// lie in memory): lse and D of the 128 rows, and for each of the P positions
+// its routing weights of the key block's chunks and the mask word holding
+// them.
+struct BwdRowInfo {
+  float lse[128];
+  float D[128];
+  float w[32][2];
+  uint32_t mword[32];
+};
+
+// Named barrier `id` over 128 threads that also ANDs a predicate across them.
+__device__ __forceinline__ bool bar_and_128(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r) : "r"((uint32_t)v), "r"(id) : "memory");
+  return r != 0;
+}
+
+template <int CHUNK>
+__global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    const BwdParams prm) {
+  constexpr int D = 128;
+  constexpr int KB = 128;                        // keys per CTA
+  constexpr int NCK = KB / CHUNK;                // chunks per key block (2 or 1)
+  constexpr int NS = 2;                          // query-tile ring depth
+  constexpr int QBOX = 128 * 128;                // 128 rows x 128 B
+  constexpr int T_BYTES = 2 * QBOX;              // one 128 x 128 bf16 tile
+  constexpr uint32_t TM_DK = 0, TM_DV = 128, TM_S = 256, TM_DP = 384;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;                            // the block's keys (two 64-column boxes)
+  uint8_t* sV = sK + T_BYTES;
+  uint8_t* sQ = sV + T_BYTES;                    // [NS] query tiles
+  uint8_t* sdO = sQ + NS * T_BYTES;              // [NS]
+  BwdRowInfo* info = reinterpret_cast<BwdRowInfo*>(sdO + NS * T_BYTES);   // [NS]
+  float2* rowtab = reinterpret_cast<float2*>(info + NS);                  // [2][NCK][128]
+
+  __shared__ __align__(8) uint64_t bar_kv, bar_full[NS], bar_empty[NS], bar_st_full, bar_p_full, bar_fin;
+  __shared__ int slot_tile[NS];
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_s;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_kb = (prm.seq + KB - 1) / KB;      // the grid's key blocks (the last may be half)
+  const int kb = (int)(blockIdx.x % n_kb);       // early key blocks (the most tiles) first
+  const int bg = (int)(blockIdx.x / n_kb);
+  const int b = bg / prm.n_kv, g = bg % prm.n_kv;
+  const int P = prm.P, G = prm.G;
+  const int kc0 = kb * NCK;                      // first chunk of the key block
+  const int key0 = kb * KB;
+
+  if (warp == 5) {
+    tmem_alloc(&tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_kv, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar_full[s], 1 + 32);           // TMA bytes + the 32 producer lanes' copies
+      mbar_init(&bar_empty[s], 1);
+    }
+    mbar_init(&bar_st_full, 1);
+    mbar_init(&bar_p_full, 128);
+    mbar_init(&bar_fin, 1);
+    abort_s = 0;
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    // K, V of the key block once; then, in position order, every query tile
+    // whose rows attend to a key of the block: the tiles of the block's own
+    // chunks (causal) and the later tiles whose routed union (written by the
+    // dQ kernel) holds one of the block's chunks.  A tile id of -1 ends it.
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar_kv, 2 * T_BYTES);
+#pragma unroll
+      for (int kb2 = 0; kb2 < 2; ++kb2) {
+        tma_load_2d(sK + kb2 * QBOX, &tmK, &bar_kv, kb2 * 64, bg * prm.seq + key0);
+        tma_load_2d(sV + kb2 * QBOX, &tmV, &bar_kv, kb2 * 64, bg * prm.seq + key0);
+      }
+    }
+    const int tile0 = key0 / P;                  // first tile of the block's chunks
+    const int tile_own = (key0 + KB) / P;        // first tile after them
+    const int wsel = kc0 >> 5;                   // mask word holding the block's chunks
+    uint32_t bsel = 0;
+#pragma unroll
+    for (int ck = 0; ck < NCK; ++ck) bsel |= 1u << ((kc0 + ck) & 31);
+    const uint32_t* tm_row = prm.tmask + ((size_t)bg * prm.nw + wsel) * prm.n_tiles;
+    int n_it = 0;                                // tiles issued
+    bool go = true;
+    for (int t0 = tile0; go && t0 < prm.n_tiles; t0 += 32) {
+      const int tt = t0 + lane;
+      const bool rel = tt < prm.n_tiles && (tt < tile_own || (__ldg(tm_row + tt) & bsel) != 0);
+      uint32_t ballot = __ballot_sync(0xffffffffu, rel);
+      while (ballot) {
+        const int bit = __ffs(ballot) - 1;
+        ballot &= ballot - 1;
+        const int tt2 = t0 + bit;
+        const int s = n_it % NS;
+        int okw = 1;
+        if (n_it >= NS && lane == 0) okw = (int)mbar_wait(&bar_empty[s], ((n_it / NS) - 1) & 1, &abort_s);
+        if (!__shfl_sync(0xffffffffu, okw, 0)) { go = false; break; }
+        const int pos_t = tt2 * P;
+        if (lane == 0) {
+          slot_tile[s] = tt2;
+          mbar_arrive_expect_tx(&bar_full[s], 2 * T_BYTES);
+#pragma unroll
+          for (int kb2 = 0; kb2 < 2; ++kb2) {
+            tma_load_3d(sQ + s * T_BYTES + kb2 * QBOX, &tmQ, &bar_full[s], kb2 * 64, b * prm.n_q + g * G, pos_t);
+            tma_load_3d(sdO + s * T_BYTES + kb2 * QBOX, &tmdO, &bar_full[s], kb2 * 64, b * prm.n_q + g * G, pos_t);
+          }
+        }
+        // lse and D: head h's P positions are contiguous (16-byte pieces)
+        BwdRowInfo* in = info + s;
+        for (int e = lane; e < 2 * G * (P / 4); e += 32) {
+          const int which = e / (G * (P / 4));
+          const int rem = e % (G * (P / 4));
+          const int h = rem / (P / 4), q4 = rem % (P / 4);
+          const size_t src = ((size_t)b * prm.n_q + g * G + h) * prm.seq + pos_t + q4 * 4;
+          cp_async_16((which ? in->D : in->lse) + h * P + q4 * 4, (which ? prm.Drow : prm.lse) + src);
+        }
+        for (int e = lane; e < P * NCK; e += 32) {
+          const int p2 = e / NCK, ck = e % NCK;
+          if (kc0 + ck < prm.n_c)                // an odd chunk count leaves a half block
+            cp_async_4(&in->w[p2][ck], prm.w + ((size_t)bg * prm.seq + pos_t + p2) * prm.n_c + kc0 + ck);
+        }
+        for (int p2 = lane; p2 < P; p2 += 32)
+          cp_async_4(&in->mword[p2], prm.mask + ((size_t)bg * prm.seq + pos_t + p2) * prm.nw + wsel);
+        cp_async_arrive_noinc(&bar_full[s]);
+        ++n_it;
+      }
+    }
+    if (go) {
+      const int s = n_it % NS;
+      int okw = 1;
+      if (n_it >= NS && lane == 0) okw = (int)mbar_wait(&bar_empty[s], ((n_it / NS) - 1) & 1, &abort_s);
+      if (__shfl_sync(0xffffffffu, okw, 0)) {
+        if (lane == 0) {
+          slot_tile[s] = -1;
+          mbar_arrive(&bar_full[s]);
+        }
+        __syncwarp();
+        mbar_arrive(&bar_full[s]);
+      }
+    }
+    if (abort_s && lane == 0) {
+      mbar_wait(&bar_kv, 0, nullptr);
+      for (int j = (n_it > NS ? n_it - NS : 0); j < n_it; ++j)
+        mbar_wait(&bar_full[j % NS], (j / NS) & 1, nullptr);
+    }
+    cp_async_wait_all();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idT = idesc_bf16_f32(128, 128, 0, 0);    // S^T, dP^T: keys x rows
+    constexpr uint32_t idA = idesc_bf16_f32(128, D, 0, 1);      // dV, dK: keys x d
+    const bool leader = elect_one();
+    const uint64_t dKk = sw128_desc(smem_u32(sK), 16, 1024);     // K, V as the K-major A
+    const uint64_t dVk = sw128_desc(smem_u32(sV), 16, 1024);
+    const uint64_t dQk0 = sw128_desc(smem_u32(sQ), 16, 1024);    // Q, dO as the K-major B
+    const uint64_t ddOk0 = sw128_desc(smem_u32(sdO), 16, 1024);
+    const uint64_t dQm0 = sw128_desc(smem_u32(sQ), QBOX, 1024);  // Q, dO as the MN-major B
+    const uint64_t ddOm0 = sw128_desc(smem_u32(sdO), QBOX, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t par) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, &abort_s));
+    };
+    bool ok = wait_all(&bar_kv, 0);
+    for (int n = 0; ok; ++n) {
+      const int s = n % NS;
+      if (!(ok = wait_all(&bar_full[s], (n / NS) & 1))) break;
+      if (slot_tile[s] < 0) break;
+      tc_fence_after();
+      const uint32_t so = (uint32_t)(s * T_BYTES);
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * QBOX + (kk & 3) * 32;
+          tc_mma_ss(tmem + TM_S, dKk + (off >> 4), dQk0 + ((so + off) >> 4), idT, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * QBOX + (kk & 3) * 32;
+          tc_mma_ss(tmem + TM_DP, dVk + (off >> 4), ddOk0 + ((so + off) >> 4), idT, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bar_st_full);
+      }
+      __syncwarp();
+      if (!(ok = wait_all(&bar_p_full, n & 1))) break;
+      tc_fence_after();
+      if (leader) {
+        // dV += P^T dO, dK += dS^T Q: K-steps of 16 query rows
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          tc_mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8, ddOm0 + ((so + kk * 2048) >> 4), idA,
+                    (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          tc_mma_ts(tmem + TM_DK, tmem + TM_DP + kk * 8, dQm0 + ((so + kk * 2048) >> 4), idA,
+                    (n > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&bar_empty[s]);
+      }
+      __syncwarp();
+    }
+    if (leader) tc_commit(&bar_fin);
+    __syncwarp();
+    if (abort_s && lane == 0) mbar_wait(&bar_fin, 0, nullptr);
+  } else {
+    // ------------------------------------------------------------ key threads (warps 0-3)
+    const int k = tid;                           // key of the block = TMEM lane
+    const int kpos = key0 + k;
+    const int kchunk = kpos / CHUNK;
+    const int ck = kchunk - kc0;                 // the key's chunk within the block
+    const uint32_t tlane = (uint32_t)((warp & 3) * 32) << 16;
+    const float scale = prm.scale_log2;
+    bool ok = mbar_wait(&bar_kv, 0, &abort_s);
+    int n = 0;
+    for (;; ++n) {
+      // every exit of this loop is taken by all 128 key threads together: the
+      // named barrier below is reached once per tile by each of them
+      const int s = n % NS;
+      const bool okw = ok && mbar_wait(&bar_full[s], (n / NS) & 1, &abort_s);
+      const int tt = okw ? slot_tile[s] : -1;
+      const BwdRowInfo* in = info + s;
+      const int pos_t = tt * P;
+      const int c_t = pos_t / CHUNK;
+      // row table of the tile (row t = p G + h): per chunk of the block the
+      // exponent offset (log2 units: routing bias minus lse; -inf where the
+      // row does not see the chunk) and D
+      float2* tab = rowtab + (n & 1) * NCK * 128;
+      if (tt >= 0) {
+        const int t = tid, pp = t >> prm.lgG, hh = t & (G - 1);
+        const int ri = hh * P + pp;
+        const float l2 = in->lse[ri] * 1.4426950408889634f;
+        const float Dv = in->D[ri];
+#pragma unroll
+        for (int c2 = 0; c2 < NCK; ++c2) {
+          const int kch = kc0 + c2;
+          float off = -INFINITY;
+          if (kch == c_t) off = -l2;
+          else if (kch < c_t && ((in->mword[pp] >> (kch & 31)) & 1u))
+            off = (prm.sigma != 0.f ? prm.sigma * lg2f(in->w[pp][c2]) : 0.f) - l2;
+          tab[c2 * 128 + t] = make_float2(off, Dv);
+        }
+      }
+      if (!bar_and_128(1, okw)) { ok = false; break; }
+      if (tt < 0) break;                         // uniform once every wait succeeded
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_st_full, n & 1, &abort_s))) {
+        ok = false;                              // the next vote ends the walk
+        continue;
+      }
+      tc_fence_after();
+      // causal on the diagonal chunk: row t sees key kpos iff its position
+      // pos_t + t / G >= kpos, i.e. t >= (kpos - pos_t) G
+      const int colmin = kchunk == c_t ? (kpos - pos_t) * G : 0;
+      const float2* tk = tab + ck * 128;
+#pragma unroll 1
+      for (int q = 0; q < 128 / 32; ++q) {
+        float sv[32], dp[32];
+        tmem_ld32(tmem + tlane + TM_S + q * 32, sv);
+        tmem_ld32(tmem + tlane + TM_DP + q * 32, dp);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int i2 = 0; i2 < 16; ++i2) {
+          float pv[2], dv2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col = q * 32 + 2 * i2 + u;
+            const float2 od = tk[col];
+            const float pr = col >= colmin ? ex2f(fmaf(sv[2 * i2 + u], scale, od.x)) : 0.f;
+            pv[u] = pr;
+            dv2[u] = pr * (dp[2 * i2 + u] - od.y);
+          }
+          pk[i2] = pack_bf16x2(pv[0], pv[1]);
+          dk[i2] = pack_bf16x2(dv2[0], dv2[1]);
+        }
+        // P^T over the S^T columns already read, dS^T over dP^T's
+        tmem_st16u(tmem + tlane + TM_S + q * 16, pk);
+        tmem_st16u(tmem + tlane + TM_DP + q * 16, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_p_full);
+    }
+    // kpos < seq is warp-uniform (seq is a multiple of 64)
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_fin, 0, &abort_s)) && kpos < prm.seq) {
+      tc_fence_after();
+      float* krow = prm.dK + ((size_t)bg * prm.seq + kpos) * D;
+      float* vrow = prm.dV + ((size_t)bg * prm.seq + kpos) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float o[32];
+        if (n > 0) {
+          tmem_ld32(tmem + tlane + TM_DK + cc * 32, o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        }
+        float4* dst = reinterpret_cast<float4*>(krow + cc * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          dst[q4] = make_float4(o[4 * q4] * prm.scale, o[4 * q4 + 1] * prm.scale,
+                                o[4 * q4 + 2] * prm.scale, o[4 * q4 + 3] * prm.scale);
+        if (n > 0) tmem_ld32(tmem + tlane + TM_DV + cc * 32, o);
+        dst = reinterpret_cast<float4*>(vrow + cc * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+inline size_t attn_bwd_dkv_smem_bytes() {
+  return (size_t)2 * 2 * 128 * 128 + (size_t)2 * 2 * 2 * 128 * 128 + 2 * sizeof(BwdRowInfo) +
+         (size_t)2 * 2 * 128 * sizeof(float2) + 1024;
+}
+
+// dQ / dw kernel, then the dK / dV kernel, on one stream (the second reads
+// the D rows and tile unions the first writes).  K / V maps: boxes of 64
+// rows (kv64) for the dQ kernel, 128 rows (kv128) for the dK / dV kernel.
+template <int CHUNK>
+cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk64,
+                               const CUtensorMap& tv64, const CUtensorMap& tk128,
+                               const CUtensorMap& tv128, const BwdParams& prm, cudaStream_t st) {
+  const size_t smem_a = attn_bwd_dq_smem_bytes(prm.n_c, prm.nw, prm.P);
+  const size_t smem_b = attn_bwd_dkv_smem_bytes();
+  auto ka = attn_bwd_dq_kernel<CHUNK>;
+  auto kb = attn_bwd_dkv_kernel<CHUNK>;
+  cudaError_t e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b);
+  if (e != cudaSuccess) return e;
+  ka<<<(unsigned)(prm.n_tiles * prm.n_bg), 192, smem_a, st>>>(tq, tdo, tk64, tv64, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int n_kb = (prm.seq + 127) / 128;
+  kb<<<(unsigned)(n_kb * prm.n_bg), 192, smem_b, st>>>(tq, tdo, tk128, tv128, prm);
+  return cudaGetLastError();
+}
+
+// Scratch of the two kernels: D rows [b, n_q, seq] fp32 and the tile unions
+// [b * n_kv, nw, seq / P] u32, each 256-byte aligned.
+inline size_t attn_bwd_tc_workspace_bytes(int batch, int n_q, int n_kv, int seq, int n_c) {
+  const int G = n_q / n_kv, P = 128 / G;
+  const size_t d_bytes = ((size_t)batch * n_q * seq * 4 + 255) & ~(size_t)255;
+  const size_t t_bytes = ((size_t)batch * n_kv * ((n_c + 31) / 32) * (seq / P) * 4 + 255) & ~(size_t)255;
+  return d_bytes + t_bytes;
+}
+
+}  // namespace dash

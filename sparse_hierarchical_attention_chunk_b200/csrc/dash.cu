@@ -18,6 +18,7 @@
 #include "route_tc.cuh"
 #include "route_topk.cuh"
 #include "attn_bwd.cuh"
+#include "attn_bwd_tc.cuh"
 #include "route_bwd.cuh"
 #include "attn_tc.cuh"
 #include "attn_f32.cuh"
@@ -106,6 +107,78 @@ int run_attn_tc(const dash_problem* p, const void* Q, const void* K, const void*
   return cuda_status(dash::launch_attn_tc<CHUNK, D>(tq, tk, tv, prm, st));
 }
 
+// Stage 2 backward on tcgen05: bf16, d = 128, G in {4, 8, 16}.
+bool attn_bwd_tc_applies(const dash_problem* p) {
+  const int G = p->n_q_heads / p->n_kv_heads;
+  return p->dtype == DASH_BF16 && p->head_dim == 128 && (G == 4 || G == 8 || G == 16);
+}
+
+size_t attn_bwd_ws_bytes(const dash_problem* p) {
+  if (!attn_bwd_tc_applies(p)) return 0;
+  return dash::attn_bwd_tc_workspace_bytes(p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len,
+                                           n_chunks(p));
+}
+
+template <int CHUNK>
+int run_attn_bwd_tc(const dash_problem* p, const void* Q, const void* K, const void* V,
+                    const float* w, const uint32_t* mask, const void* O, const float* lse,
+                    const void* dO, float* dQ, float* dK, float* dV, float* dw, void* workspace,
+                    cudaStream_t st) {
+  constexpr uint64_t d = 128;
+  const int G = p->n_q_heads / p->n_kv_heads;
+  const int P = 128 / G;
+  CUtensorMap tq, tdo, tk64, tv64, tk128, tv128;
+  {
+    // Q and dO viewed as (d, head, position): a box {64, G, P} lands
+    // position-major, shared-memory row r = p * G + h
+    const uint64_t dims[3] = {d, (uint64_t)p->batch * p->n_q_heads, (uint64_t)p->seq_len};
+    const uint64_t str[2] = {(uint64_t)p->seq_len * d * 2, d * 2};
+    const uint32_t box[3] = {64, (uint32_t)G, (uint32_t)P};
+    if (!make_tmap(&tq, Q, 3, dims, str, box)) return DASH_ERR_CUDA;
+    if (!make_tmap(&tdo, dO, 3, dims, str, box)) return DASH_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[2] = {d, (uint64_t)p->batch * p->n_kv_heads * p->seq_len};
+    const uint64_t str[1] = {d * 2};
+    const uint32_t box64[2] = {64, 64}, box128[2] = {64, 128};
+    if (!make_tmap(&tk64, K, 2, dims, str, box64) || !make_tmap(&tv64, V, 2, dims, str, box64) ||
+        !make_tmap(&tk128, K, 2, dims, str, box128) || !make_tmap(&tv128, V, 2, dims, str, box128))
+      return DASH_ERR_CUDA;
+  }
+  dash::BwdParams prm;
+  prm.w = w;
+  prm.mask = mask;
+  prm.lse = lse;
+  prm.O = static_cast<const bf16*>(O);
+  prm.dO = static_cast<const bf16*>(dO);
+  prm.dQ = dQ;
+  prm.dK = dK;
+  prm.dV = dV;
+  prm.dw = dw;
+  prm.n_q = p->n_q_heads;
+  prm.n_kv = p->n_kv_heads;
+  prm.seq = p->seq_len;
+  prm.chunk = p->chunk;
+  prm.n_c = n_chunks(p);
+  prm.nw = (prm.n_c + 31) / 32;
+  prm.G = G;
+  prm.lgG = G == 4 ? 2 : G == 8 ? 3 : 4;
+  prm.P = P;
+  prm.n_tiles = p->seq_len / P;
+  prm.n_bg = p->batch * p->n_kv_heads;
+  prm.sigma = p->sigma;
+  prm.scale = 1.f / sqrtf((float)d);
+  prm.scale_log2 = 1.4426950408889634f * prm.scale;
+  const size_t d_bytes = ((size_t)p->batch * p->n_q_heads * p->seq_len * 4 + 255) & ~(size_t)255;
+  prm.Drow = static_cast<float*>(workspace);
+  prm.tmask = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + d_bytes);
+  if (dw) {
+    const cudaError_t e = cudaMemsetAsync(dw, 0, (size_t)prm.n_bg * p->seq_len * prm.n_c * sizeof(float), st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return cuda_status(dash::launch_attn_bwd_tc<CHUNK>(tq, tdo, tk64, tv64, tk128, tv128, prm, st));
+}
+
 }  // namespace
 
 extern "C" {
@@ -122,7 +195,7 @@ const char* dash_status_str(int s) {
   }
 }
 
-int dash_version(void) { return (2 << 16) | 0; }
+int dash_version(void) { return (3 << 16) | 0; }
 
 int dash_summarize(const dash_problem* p, const void* K, const float* qbar, int chunk_begin,
                    int chunk_end, void* Kbar, void* stream) {
@@ -200,7 +273,8 @@ int dash_route_topk(const dash_problem* p, const void* Q, const void* Kbar, int 
 
 int dash_attn_bwd(const dash_problem* p, const void* Q, const void* K, const void* V,
                   const float* w, const uint32_t* mask, const void* O, const float* lse,
-                  const void* dO, float* dQ, float* dK, float* dV, float* dw, void* stream) {
+                  const void* dO, float* dQ, float* dK, float* dV, float* dw, void* workspace,
+                  size_t workspace_bytes, void* stream) {
   int rc = check_problem(p, false);
   if (rc) return rc;
   const void* req[] = {Q, K, V, w, mask, O, lse, dO, dQ, dK, dV};
@@ -209,6 +283,14 @@ int dash_attn_bwd(const dash_problem* p, const void* Q, const void* K, const voi
   if (dw && !aligned16(dw)) return DASH_ERR_INVALID_ARG;
   if (p->n_q_heads / p->n_kv_heads > 16) return DASH_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (attn_bwd_tc_applies(p)) {
+    const size_t need = attn_bwd_ws_bytes(p);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return DASH_ERR_WORKSPACE;
+    return p->chunk == 64
+               ? run_attn_bwd_tc<64>(p, Q, K, V, w, mask, O, lse, dO, dQ, dK, dV, dw, workspace, st)
+               : run_attn_bwd_tc<128>(p, Q, K, V, w, mask, O, lse, dO, dQ, dK, dV, dw, workspace, st);
+  }
   const size_t kv_bytes = (size_t)p->batch * p->n_kv_heads * p->seq_len * p->head_dim * sizeof(float);
   cudaError_t e = cudaMemsetAsync(dK, 0, kv_bytes, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(dV, 0, kv_bytes, st);
@@ -322,9 +404,11 @@ int dash_route_packed(const dash_problem* p, const void* Q, const void* Kbar, co
   return route_entry(p, Q, Kbar, K, qbar, weight, mask, true, count, index, stream);
 }
 
-size_t dash_workspace_bytes(const dash_problem* p, int is_decode) {
-  if (check_problem(p, is_decode != 0) != DASH_OK) return 0;
-  if (!is_decode) return 0;
+size_t dash_workspace_bytes(const dash_problem* p, int which) {
+  if (which < 0 || which > 2) return 0;
+  if (check_problem(p, which == 1) != DASH_OK) return 0;
+  if (which == 0) return 0;
+  if (which == 2) return attn_bwd_ws_bytes(p);
   return dash::decode_workspace_bytes(p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len,
                                       p->head_dim, p->chunk);
 }

@@ -84,7 +84,7 @@ def lib():
         L.dash_summarize_bwd.restype = i32
         L.dash_summarize_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp]
         L.dash_attn_bwd.restype = i32
-        L.dash_attn_bwd.argtypes = [P] + [vp] * 13
+        L.dash_attn_bwd.argtypes = [P] + [vp] * 13 + [ctypes.c_size_t, vp]
         L.dash_route.restype = i32
         L.dash_route.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.dash_route_packed.restype = i32
@@ -216,8 +216,10 @@ def dash_route_topk(p, Q, Kbar, k, w, mask, stream=None):
                                                     _ptr(w), _ptr(mask), _stream(stream)))
 
 
-def dash_attn_bwd(p, Q, K, V, w, mask, O, lse, dO, dQ, dK, dV, dw=None, stream=None):
-    """Stage-2 gradients (fp32 dQ, dK, dV, and dw if given) for the cotangent dO."""
+def dash_attn_bwd(p, Q, K, V, w, mask, O, lse, dO, dQ, dK, dV, dw=None, workspace=None, stream=None):
+    """Stage-2 gradients (fp32 dQ, dK, dV, and dw if given) for the cotangent dO.
+    `workspace` (uint8, dash_workspace_bytes(p, 2) bytes) is allocated here
+    when not given."""
     dt = _tdtype(p)
     f32 = torch.float32
     _check(Q, "Q", (p.batch, p.n_q_heads, p.seq_len, p.head_dim), dt)
@@ -233,9 +235,14 @@ def dash_attn_bwd(p, Q, K, V, w, mask, O, lse, dO, dQ, dK, dV, dw=None, stream=N
     _check(dV, "dV", (p.batch, p.n_kv_heads, p.seq_len, p.head_dim), f32)
     if dw is not None:
         _check(dw, "dw", (p.batch, p.n_kv_heads, p.seq_len, n_chunks(p)), f32)
+    need = dash_workspace_bytes(p, 2)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _raise("dash_attn_bwd", lib().dash_attn_bwd(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(w),
                                                 _ptr(mask), _ptr(O), _ptr(lse), _ptr(dO), _ptr(dQ),
-                                                _ptr(dK), _ptr(dV), _ptr(dw), _stream(stream)))
+                                                _ptr(dK), _ptr(dV), _ptr(dw), _ptr(workspace),
+                                                ws_bytes, _stream(stream)))
 
 
 def dash_route_bwd(p, Q, Kbar, dw, dQ, dKbar, stream=None):
@@ -271,7 +278,8 @@ def backward(p, Q, K, V, qbar, out, dO, stream=None):
     dw = torch.empty(out["w"].shape, **f32)
     dKbar = torch.zeros(out["Kbar"].shape, **f32)
     dqbar = torch.zeros(qbar.shape, **f32)
-    dash_attn_bwd(p, Q, K, V, out["w"], out["mask"], out["O"], out["lse"], dO, dQ, dK, dV, dw, stream)
+    dash_attn_bwd(p, Q, K, V, out["w"], out["mask"], out["O"], out["lse"], dO, dQ, dK, dV, dw,
+                  stream=stream)
     dash_route_bwd(p, Q, out["Kbar"], dw, dQ, dKbar, stream)
     dash_summarize_bwd(p, K, qbar, dKbar, dK, dqbar, stream)
     return {"dQ": dQ, "dK": dK, "dV": dV, "dqbar": dqbar, "dw": dw, "dKbar": dKbar}
@@ -336,8 +344,10 @@ def dash_attn_fwd_packed(p, Q, K, V, weight, mask, O, lse=None, stream=None):
                                       _ptr(mask), _ptr(O), _ptr(lse), _stream(stream)))
 
 
-def dash_workspace_bytes(p, is_decode):
-    return int(lib().dash_workspace_bytes(ctypes.byref(p), 1 if is_decode else 0))
+def dash_workspace_bytes(p, which):
+    """Scratch bytes of dash_attn_fwd (which = 0 or False), the decode entry
+    points (1 or True) or dash_attn_bwd (2)."""
+    return int(lib().dash_workspace_bytes(ctypes.byref(p), int(which)))
 
 
 def dash_attn_fwd(p, Q, K, V, w, mask, O, lse=None, workspace=None, stream=None):

@@ -38,7 +38,7 @@ def test_status_strings_and_version(L):
     assert dash.status_str(0) == "DASH_OK"
     assert dash.status_str(4) == "DASH_ERR_TIMEOUT"
     assert dash.status_str(99) == "DASH_ERR_UNKNOWN"
-    assert L.dash_version() >> 16 == 2
+    assert L.dash_version() >> 16 == 3
 
 
 def _p(**kw):
@@ -147,9 +147,26 @@ def test_attn_bwd_arguments_checked(L):
     for k in range(11):                                # every required pointer
         a = list(args)
         a[k] = None
-        assert L.dash_attn_bwd(ctypes.byref(p), *a, None, None) == dash.DASH_ERR_INVALID_ARG
+        assert L.dash_attn_bwd(ctypes.byref(p), *a, None, None, 0, None) == dash.DASH_ERR_INVALID_ARG
     odd = ctypes.c_void_p((1 << 20) + 8)
-    assert L.dash_attn_bwd(ctypes.byref(p), *args, odd, None) == dash.DASH_ERR_INVALID_ARG
+    assert L.dash_attn_bwd(ctypes.byref(p), *args, odd, None, 0, None) == dash.DASH_ERR_INVALID_ARG
+
+
+@host_only
+def test_attn_bwd_workspace_checked(L):
+    # the tensor-core backward (bf16, d = 128, G in {4, 8, 16}) needs scratch
+    # for its D rows and tile unions; the reference kernel needs none
+    p = _p()
+    need = dash.dash_workspace_bytes(p, 2)
+    assert need == 1 * 32 * 1024 * 4 + ((1 * 2 * 1 * (1024 // 8) * 4 + 255) // 256) * 256
+    assert dash.dash_workspace_bytes(_p(dtype="f32"), 2) == 0
+    assert dash.dash_workspace_bytes(_p(head_dim=64), 2) == 0
+    assert dash.dash_workspace_bytes(p, 3) == 0
+    args = [FAKE] * 11
+    assert L.dash_attn_bwd(ctypes.byref(p), *args, None, None, need, None) == dash.DASH_ERR_WORKSPACE
+    assert L.dash_attn_bwd(ctypes.byref(p), *args, None, FAKE, need - 1, None) == dash.DASH_ERR_WORKSPACE
+    odd = ctypes.c_void_p((1 << 20) + 16)
+    assert L.dash_attn_bwd(ctypes.byref(p), *args, None, odd, need, None) == dash.DASH_ERR_WORKSPACE
 
 
 @host_only

@@ -898,9 +898,17 @@ def test_attention_on_topk_mask_matches_oracle():
 # ----------------------------------------------------------------------------
 
 BWD = {
+    # CUDA-core reference kernel
     "tiny_f32": (configs.TINY_F32, 1e-4),
     "g8_d64_b64_batch2": (MED["g8_d64_b64_batch2"], 2e-2),
+    # tcgen05 kernels: an odd chunk count (a half key block at the end), 128-key
+    # chunks with sigma = 0.5, G = 4 with sigma = 0 (no dw), G = 8 over two
+    # sequences
     "g16_d128_b64_nc37": (MED["g16_d128_b64_nc37"], 2e-2),
+    "g16_d128_b128_s05": (MED["g16_d128_b128_s05"], 2e-2),
+    "g4_d128_sigma0": (MED["g4_d128_sigma0"], 2e-2),
+    "g8_d128_b128_batch2": (W("med_g8_d128", "prefill", 2, 16, 2, 12 * 128, 128, 128, sigma=1.0,
+                              rho=(0.9, 0.5), needles=(2, 1)), 2e-2),
 }
 
 
@@ -931,6 +939,83 @@ def test_attn_bwd_matches_oracle(name):
     # dw lives only on the active routed blocks
     act = oracle.unpack_mask(mask_from_dev(out["mask"]), wl.n_chunks)
     assert not np64(dw)[~act].any()
+
+
+def test_attn_bwd_tc_is_deterministic():
+    # every output element is written once, in a fixed order: two calls agree bit for bit
+    wl = BWD["g16_d128_b64_nc37"][0]
+    inp = synth.make_prefill(wl, seed=32)
+    p = dash.problem_for(wl)
+    assert dash.dash_workspace_bytes(p, 2) > 0
+    dev = {n: inp[n].cuda() for n in ("Q", "K", "V", "qbar")}
+    out = dash.prefill(p, dev["Q"], dev["K"], dev["V"], dev["qbar"])
+    dO = torch.randn(dev["Q"].shape, generator=torch.Generator().manual_seed(33)).to(torch.bfloat16).cuda()
+    f32 = dict(dtype=torch.float32, device="cuda")
+    res = []
+    for _ in range(2):
+        g = [torch.empty(dev["Q"].shape, **f32), torch.empty(dev["K"].shape, **f32),
+             torch.empty(dev["V"].shape, **f32), torch.empty(out["w"].shape, **f32)]
+        dash.dash_attn_bwd(p, dev["Q"], dev["K"], dev["V"], out["w"], out["mask"], out["O"], out["lse"],
+                           dO, *g)
+        res.append(g)
+    assert dash.dash_get_error() == dash.DASH_OK
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
+
+
+def test_attn_bwd_workspace_checked():
+    wl = BWD["g16_d128_b64_nc37"][0]
+    p = dash.problem_for(wl)
+    need = dash.dash_workspace_bytes(p, 2)
+    Q = torch.zeros(wl.batch, wl.n_q_heads, wl.seq, wl.head_dim, dtype=torch.bfloat16, device="cuda")
+    K = torch.zeros(wl.batch, wl.n_kv_heads, wl.seq, wl.head_dim, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(wl.batch, wl.n_kv_heads, wl.seq, wl.n_chunks, device="cuda")
+    m = torch.zeros(wl.batch, wl.n_kv_heads, wl.seq, (wl.n_chunks + 31) // 32, dtype=torch.int32, device="cuda")
+    lse = torch.zeros(wl.batch, wl.n_q_heads, wl.seq, device="cuda")
+    dQ, dK = Q.float(), K.float()
+    short = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(RuntimeError, match="DASH_ERR_WORKSPACE"):
+        dash.dash_attn_bwd(p, Q, K, K, w, m, Q, lse, Q, dQ, dK, dK.clone(), workspace=short)
+
+
+def test_attn_bwd_full_size_8k():
+    # the bench's backward workload (8k, G = 16, 64-key chunks) in the same
+    # launch: dQ and dw of sampled positions against the oracle row by row;
+    # dK and dV through identities that hold at any size -- summed over the
+    # keys, dV equals the group's dO summed over its rows (each row's p sums
+    # to 1) and dK vanishes (each row's ds sums to 0)
+    from oracle import dash_oracle_bwd as obwd
+    wl = configs.PREFILL_8K
+    inp = synth.make_prefill(wl, seed=34, device="cuda")
+    p = dash.problem_for(wl)
+    out = dash.prefill(p, inp["Q"], inp["K"], inp["V"], inp["qbar"])
+    dO = torch.randn(inp["Q"].shape, generator=torch.Generator(device="cuda").manual_seed(35),
+                     device="cuda").to(torch.bfloat16)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    dQ, dK, dV = (torch.empty(inp[n].shape, **f32) for n in ("Q", "K", "V"))
+    dw = torch.empty(out["w"].shape, **f32)
+    dash.dash_attn_bwd(p, inp["Q"], inp["K"], inp["V"], out["w"], out["mask"], out["O"], out["lse"],
+                       dO, dQ, dK, dV, dw)
+    assert dash.dash_get_error() == dash.DASH_OK
+    pos = np.sort(np.random.default_rng(36).choice(wl.seq, 48, replace=False))
+    pos = np.unique(np.concatenate([pos, [0, 63, 64, wl.seq - 1]]))
+    m = mask_from_dev(out["mask"])[:, :, pos]
+    w = np64(out["w"])[:, :, pos]
+    dO64 = np64(dO)
+    rq, _, _, rdw = obwd.attn_bwd(np64(inp["Q"]), np64(inp["K"]), np64(inp["V"]), w, m, wl.sigma,
+                                  wl.chunk, dO64[:, :, pos], positions=pos)
+    gq = np64(dQ)[:, :, pos]
+    assert np.abs(gq - rq[:, :, pos]).max() / np.abs(rq[:, :, pos]).max() <= 2e-2
+    gdw = np64(dw)[:, :, pos]
+    assert np.abs(gdw - rdw).max() / max(np.abs(rdw).max(), 1e-30) <= 2e-2
+    G = wl.n_q_heads // wl.n_kv_heads
+    want_v = dO64.reshape(wl.batch, wl.n_kv_heads, G * wl.seq, wl.head_dim).sum(axis=2)
+    got_v = np64(dV).sum(axis=2)
+    assert np.abs(got_v - want_v).max() <= 2e-2 * np.abs(want_v).max()
+    # dK: the row sums of ds vanish up to O's bf16 rounding in D = dO . O
+    got_k = np.abs(np64(dK).sum(axis=2)).max()
+    assert got_k <= 2e-2 * np.abs(np64(dK)).sum(axis=2).max()
+    assert np.isfinite(np64(dK)).all() and np.isfinite(np64(dV)).all()
 
 
 RBWD = {
