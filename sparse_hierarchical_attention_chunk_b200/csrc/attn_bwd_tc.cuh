@@ -50,31 +50,70 @@ struct BwdParams {
   float* dw;             // nullable
   float* Drow;           // [b, n_q, seq]: dO . O (written by the dQ kernel)
   uint32_t* tmask;       // [b * n_kv, nw, n_tiles]: each tile's routed union (dQ kernel)
-  int n_q, n_kv, seq, chunk, n_c, nw, G, lgG, P, n_tiles, n_bg;
+  float* part;           // [n_split, b * n_kv * seq, 256]: partial dK | dV (n_split > 1)
+  int n_q, n_kv, seq, chunk, n_c, nw, G, lgG, P, n_tiles, n_bg, n_split;
   float sigma, scale_log2, scale;
 };
 
 // ---------------------------------------------------------------------------
 // dQ and dw
 // ---------------------------------------------------------------------------
+// K / V ring depth of the dQ kernel: block n + 2's S and dP are issued right
+// after block n's dQ, so its slot must have been freed two steps earlier
+constexpr int kBwdDqStages = 4;
+
+// Eight row warps: two per TMEM lane quarter, each taking 32 of a block's 64
+// keys; then the producer and the MMA issuer.
+constexpr int kBwdRowWarps = 8;
+
+// Two 32-column TMEM loads (32 lanes x 32-bit) and one wait, in one asm
+// statement so that no use of the registers is scheduled before the data.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float (&va)[32], float (&vb)[32]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(ta), "r"(tb)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    va[i] = __uint_as_float(r[i]);
+    vb[i] = __uint_as_float(r[32 + i]);
+  }
+}
+
 template <int CHUNK>
-__global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
+__global__ void __launch_bounds__(32 * (kBwdRowWarps + 2), 1) attn_bwd_dq_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const BwdParams prm) {
   constexpr int D = 128;
   constexpr int BLK = 64;                        // keys per block
   constexpr int SB = CHUNK / BLK;                // sub-blocks per chunk
-  constexpr int NS = 3;                          // K / V ring depth
+  constexpr int NS = kBwdDqStages;               // K / V ring depth
   constexpr int QBOX = 128 * 128;                // 128 rows x 128 B
   constexpr int T_BYTES = 2 * QBOX;              // one 128 x 128 bf16 tile
   constexpr int KV_BOX = BLK * 128;
   constexpr int KV_BYTES = 2 * KV_BOX;
   // TMEM columns: Q | dO (bf16 pairs) | dQ (fp32) | S, dP of buffer 0 | of buffer 1
   constexpr uint32_t TM_Q = 0, TM_DO = 64, TM_DQ = 128, TM_BUF = 256;
+  constexpr int NRT = 32 * kBwdRowWarps;         // row threads
+  constexpr int W_PROD = kBwdRowWarps, W_MMA = kBwdRowWarps + 1;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned by pointer arithmetic on the shared array, so that the
+  // compiler keeps the shared address space (and emits shared loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem;
   uint8_t* sdO = sQ + T_BYTES;
   uint8_t* sK = sdO + T_BYTES;
@@ -84,6 +123,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
   float* w_sm = reinterpret_cast<float*>(mrows + prm.P * prm.nw);        // [NS][P]
 
   __shared__ __align__(8) uint64_t bar_qd, bar_qd_tm, bar_s_full[2], bar_ds_full[2], bar_fin;
+  __shared__ float dpart[2][128];                // the halves of each row's dO . O
   __shared__ __align__(8) uint64_t bar_k_full[NS], bar_k_empty[NS], bar_v_full[NS], bar_v_empty[NS];
   __shared__ uint32_t tmem_slot;
   __shared__ int nb_s;
@@ -98,16 +138,16 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
   const int c_i = pos0 / CHUNK;
   const int n_wl = min(P, 32);
 
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tmem_alloc(&tmem_slot, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
     mbar_init(&bar_qd, 1);
-    mbar_init(&bar_qd_tm, 128);
+    mbar_init(&bar_qd_tm, NRT);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar_s_full[t], 1);
-      mbar_init(&bar_ds_full[t], 128);
+      mbar_init(&bar_ds_full[t], NRT);
     }
     mbar_init(&bar_fin, 1);
     for (int s = 0; s < NS; ++s) {
@@ -176,7 +216,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
     return e;
   };
 
-  if (warp == 4) {
+  if (warp == W_PROD) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar_qd, 2 * T_BYTES);
@@ -225,7 +265,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
       }
       cp_async_wait_all();
     }
-  } else if (warp == 5) {
+  } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer
     // S(n), dP(n) into buffer n & 1; after block n's dS: dQ(n), then S(n+2),
     // dP(n+2) into the same buffer (in issue order, after dQ(n) read dS(n)).
@@ -275,9 +315,10 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
       const uint32_t ds = tmem + TM_BUF + (uint32_t)(n & 1) * 128;   // dS(n), bf16 pairs
       const uint64_t dkm = dKmn0 + (uint64_t)((s * KV_BYTES) >> 4);
       if (leader) {
+        // dS of keys 32 h + 16 j .. (packed) sits at columns 32 h + 8 j
 #pragma unroll
         for (int kk = 0; kk < BLK / 16; ++kk)
-          tc_mma_ts(tmem + TM_DQ, ds + kk * 8, dkm + (uint64_t)((kk * 2048) >> 4), idQ,
+          tc_mma_ts(tmem + TM_DQ, ds + (kk >> 1) * 32 + (kk & 1) * 8, dkm + (uint64_t)((kk * 2048) >> 4), idQ,
                     (n > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&bar_k_empty[s]);
         tc_commit(&bar_v_empty[s]);
@@ -299,66 +340,65 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
       if (n_q > 0) mbar_wait(&bar_k_empty[(n_q - 1) % NS], ((n_q - 1) / NS) & 1, nullptr);
     }
   } else {
-    // ------------------------------------------------------------ rows (warps 0-3)
-    const int r = tid;                         // row = TMEM lane
+    // ------------------------------------------------------------ rows (warps 0-7)
+    const int r = tid & 127;                   // row = TMEM lane
+    const int half = warp >> 2;                // keys 32 half .. 32 half + 31 of each block
     const int p = r / G, hq = r % G;
     const int pos = pos0 + p;
     const int qh = g * G + hq;
     const uint32_t tlane = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t* mrow = mrows + p * prm.nw;
     const size_t qrow = ((size_t)b * prm.n_q + qh) * prm.seq + pos;
-    const float scale = prm.scale_log2, sigma = prm.sigma;
+    const float sigma = prm.sigma;
     const float lse2 = prm.lse[qrow] * 1.4426950408889634f;
-    // D = dO . O of this row (fp32), also kept for the key-major kernel
-    float Dr = 0.f;
+    const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
+    // D = dO . O of this row (fp32; each half takes 64 of the d columns), also
+    // kept for the key-major kernel
     {
-      const uint4* orow = reinterpret_cast<const uint4*>(prm.O + qrow * D);
-      const uint4* drow = reinterpret_cast<const uint4*>(prm.dO + qrow * D);
+      float dpp = 0.f;
+      const uint4* orow = reinterpret_cast<const uint4*>(prm.O + qrow * D + half * 64);
+      const uint4* drow = reinterpret_cast<const uint4*>(prm.dO + qrow * D + half * 64);
 #pragma unroll 4
-      for (int v = 0; v < D / 8; ++v) {
+      for (int v = 0; v < 8; ++v) {
         const uint4 a = __ldg(orow + v), c = __ldg(drow + v);
         const __nv_bfloat16* xa = reinterpret_cast<const __nv_bfloat16*>(&a);
         const __nv_bfloat16* xc = reinterpret_cast<const __nv_bfloat16*>(&c);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) Dr = fmaf(__bfloat162float(xa[e]), __bfloat162float(xc[e]), Dr);
+        for (int e = 0; e < 8; ++e) dpp = fmaf(__bfloat162float(xa[e]), __bfloat162float(xc[e]), dpp);
       }
-      prm.Drow[qrow] = Dr;
+      dpart[half][r] = dpp;
     }
+    asm volatile("bar.sync 1, %0;" ::"r"(NRT) : "memory");
+    const float Dr = dpart[0][r] + dpart[1][r];
+    if (half == 0) prm.Drow[qrow] = Dr;
     // waits are made warp-uniform: the TMEM loads / stores and shuffles below
     // are warp-collective
     bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_qd, 0, &abort_s));
-    // Q and dO rows: shared memory (TMA, 128-byte swizzle) -> TMEM as bf16 pairs
+    // Q (half 0) and dO (half 1) rows: shared memory (TMA, 128-byte swizzle)
+    // -> TMEM as bf16 pairs
     if (ok) {
+      const uint8_t* base = (half ? sdO : sQ) + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint8_t* base = (which ? sdO : sQ) + (r >> 3) * 1024 + (r & 7) * 128;
+      for (int kb = 0; kb < 2; ++kb) {
+        uint32_t h0[16], h1[16];
 #pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-          uint32_t v[32];
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const uint4 q4 = *reinterpret_cast<const uint4*>(base + kb * QBOX + ((ch ^ (r & 7)) << 4));
-            v[ch * 4 + 0] = q4.x;
-            v[ch * 4 + 1] = q4.y;
-            v[ch * 4 + 2] = q4.z;
-            v[ch * 4 + 3] = q4.w;
-          }
-          uint32_t h0[16], h1[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            h0[i] = v[i];
-            h1[i] = v[16 + i];
-          }
-          const uint32_t dst = tmem + tlane + (which ? TM_DO : TM_Q) + kb * 32;
-          tmem_st16u(dst, h0);
-          tmem_st16u(dst + 16, h1);
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 q4 = *reinterpret_cast<const uint4*>(base + kb * QBOX + ((ch ^ (r & 7)) << 4));
+          uint32_t* dst = ch < 4 ? h0 + ch * 4 : h1 + (ch - 4) * 4;
+          dst[0] = q4.x;
+          dst[1] = q4.y;
+          dst[2] = q4.z;
+          dst[3] = q4.w;
         }
+        const uint32_t dst = tmem + tlane + (half ? TM_DO : TM_Q) + kb * 32;
+        tmem_st16u(dst, h0);
+        tmem_st16u(dst + 16, h1);
       }
       tmem_wait_st();
     }
     tc_fence_before();
     mbar_arrive(&bar_qd_tm);
-    float dsum_chunk = 0.f;                    // dS summed over a routed chunk's sub-blocks
+    float dsum_chunk = 0.f;                    // this half's dS summed over a routed chunk
     for (int n = 0; ok && n < nbb; ++n) {
       const Entry en = entry(n);
       const int c = en.c;
@@ -383,65 +423,72 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
           if (sigma != 0.f) bias = sigma * lg2f(wc);
         }
       }
-      const uint32_t tb = tmem + tlane + TM_BUF + (uint32_t)(n & 1) * 128;
+      const uint32_t tb = tmem + tlane + TM_BUF + (uint32_t)(n & 1) * 128 + half * 32;
       float dsum = 0.f;
       if (!__any_sync(0xffffffffu, act)) {
         uint32_t z[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) z[i] = 0u;
         tmem_st16u(tb, z);
-        tmem_st16u(tb + 16, z);
       } else {
-        float sv[64], dp[64];
-        tmem_ld64(tb, sv);
-        tmem_ld64(tb + 64, dp);
-        const int lim = en.j == 0 ? pos - (c * CHUNK + en.sb * BLK) : BLK;   // causal on the diagonal
-        const float off = bias - lse2;
-        uint32_t pk[32];
+        float sv[32], dp[32];
+        tmem_ld32x2(tb, tb + 64, sv, dp);
+        // causal on the diagonal: key k of the block is seen iff k <= lim
+        const int lim = (en.j == 0 ? pos - (c * CHUNK + en.sb * BLK) : BLK) - half * 32;
+        const uint64_t off2 = f2_pack(bias - lse2, bias - lse2);
+        const uint64_t D2 = f2_pack(Dr, Dr);
+        // p = 2^(s * scale + off): 3 of every 8 pairs on the FMA pipe
+        // (exp2_poly2), the rest on the special-function unit
+        constexpr uint32_t kPolyPairs = 0x52u;   // pairs 1, 4, 6 of each 8
+        uint32_t pk[16];
 #pragma unroll
-        for (int k2 = 0; k2 < 32; ++k2) {
-          float d2[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int k = 2 * k2 + u;
-            const float pr = k <= lim ? ex2f(fmaf(sv[k], scale, off)) : 0.f;
-            d2[u] = pr * (dp[k] - Dr);
-            dsum += d2[u];
+        for (int k2 = 0; k2 < 16; ++k2) {
+          const uint64_t x = f2_fma(f2_pack(sv[2 * k2], sv[2 * k2 + 1]), sc2, off2);
+          float e0, e1;
+          if ((kPolyPairs >> (k2 & 7)) & 1u) {
+            exp2_poly2(x, e0, e1);
+          } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            e0 = ex2f(x0);
+            e1 = ex2f(x1);
           }
-          pk[k2] = pack_bf16x2(d2[0], d2[1]);
+          e0 = 2 * k2 <= lim ? e0 : 0.f;
+          e1 = 2 * k2 + 1 <= lim ? e1 : 0.f;
+          const uint64_t d2 = f2_mul(f2_pack(e0, e1), f2_sub(f2_pack(dp[2 * k2], dp[2 * k2 + 1]), D2));
+          float a0, a1;
+          f2_unpack(d2, a0, a1);
+          dsum += a0 + a1;
+          pk[k2] = pack_bf16x2(a0, a1);
         }
-        uint32_t h0[16], h1[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          h0[i] = pk[i];
-          h1[i] = pk[16 + i];
-        }
-        tmem_st16u(tb, h0);
-        tmem_st16u(tb + 16, h1);
+        tmem_st16u(tb, pk);                    // dS over the half's own S columns
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_ds_full[n & 1]);
       // dw of a routed chunk: sigma / w times the sum of dS over its keys and
-      // the heads of the position (adjacent lanes), written once per chunk
+      // the heads of the position (adjacent lanes); the two halves' shares
+      // are added to the zeroed dw (two terms: the sum does not depend on
+      // their order)
       if (en.j > 0 && prm.dw && sigma != 0.f) {
         dsum_chunk += dsum;
         if (en.sb == SB - 1) {
           float tot = dsum_chunk;
           for (int o = 1; o < G; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-          if (hq == 0 && act)
-            prm.dw[((size_t)bg * prm.seq + pos) * prm.n_c + c] = wc > 0.f ? sigma / wc * tot : 0.f;
+          if (hq == 0 && act && wc > 0.f)
+            atomicAdd(prm.dw + ((size_t)bg * prm.seq + pos) * prm.n_c + c, sigma / wc * tot);
           dsum_chunk = 0.f;
         }
       }
     }
+    // dQ: half 0 writes columns 0-63, half 1 columns 64-127
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_fin, 0, &abort_s))) {
       tc_fence_after();
-      float* drow = prm.dQ + qrow * D;
+      float* drow = prm.dQ + qrow * D + half * 64;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         float o[32];
-        tmem_ld32(tmem + tlane + TM_DQ + cc * 32, o);
+        tmem_ld32(tmem + tlane + TM_DQ + half * 64 + cc * 32, o);
         float4* dst = reinterpret_cast<float4*>(drow + cc * 32);
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4)
@@ -452,80 +499,117 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
 inline size_t attn_bwd_dq_smem_bytes(int n_c, int nw, int P) {
-  return (size_t)2 * 2 * 128 * 128 + (size_t)3 * 2 * 2 * 64 * 128 + (size_t)(n_c + 1) * 4 +
-         (size_t)P * nw * 4 + (size_t)3 * P * 4 + 1024 + 64;
+  return (size_t)2 * 2 * 128 * 128 + (size_t)kBwdDqStages * 2 * 2 * 64 * 128 + (size_t)(n_c + 1) * 4 +
+         (size_t)P * nw * 4 + (size_t)kBwdDqStages * P * 4 + 1024 + 64;
 }
 
 // ---------------------------------------------------------------------------
 // dK and dV
 // ---------------------------------------------------------------------------
-// Per-tile row data staged beside the tile's Q and dO (head-major, as they
-// lie in memory): lse and D of the 128 rows, and for each of the P positions
-// its routing weights of the key block's chunks and the mask word holding
-// them.
-struct BwdRowInfo {
-  float lse[128];
-  float D[128];
-  float w[32][2];
-  uint32_t mword[32];
-};
 
-// Named barrier `id` over 128 threads that also ANDs a predicate across them.
-__device__ __forceinline__ bool bar_and_128(int id, bool v) {
+// Named barrier `id` over `count` threads that also ANDs a predicate across them.
+__device__ __forceinline__ bool bar_and(int id, int count, bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r) : "r"((uint32_t)v), "r"(id) : "memory");
+      : "=r"(r) : "r"((uint32_t)v), "r"(id), "r"(count) : "memory");
   return r != 0;
 }
 
+// Per 128-key CTA and 128-row query tile, in the tensor core's order:
+//   S^T(n) = K Q^T, dP^T(n) = V dO^T   (SS-MMAs, N = 128)
+//   dV += P^T(n) dO                      once the key threads wrote P^T over S^T
+//   S^T(n + 1)                           over P^T, behind dV(n)
+//   dK += dS^T(n) Q                      once they wrote dS^T over dP^T
+//   dP^T(n + 1)                          over dS^T, behind dK(n)
+// so the key threads form P^T(n + 1) while the tensor core runs dK(n) and
+// dP^T(n + 1), and dS^T(n) while it runs dV(n) and S^T(n + 1).  Eight key
+// warps: two per TMEM lane quarter, each taking 64 of the tile's 128 rows;
+// each keeps its P in registers between the two passes.
+constexpr int kBwdDkvStages = 2;                 // query-tile ring depth
+constexpr int kBwdKeyWarps = 8;
+// A key block's tile list is split over n_split CTAs (interleaved by tile
+// ordinal) when there are few key blocks: about four waves of 148 SMs.
+constexpr int kBwdSplitTarget = 4 * 148;
+constexpr int kBwdMaxSplit = 8;
+
+inline int attn_bwd_n_split(int n_kb, int n_bg) {
+  const int units = n_kb * n_bg;
+  int s = (kBwdSplitTarget + units - 1) / units;
+  return s < 1 ? 1 : (s > kBwdMaxSplit ? kBwdMaxSplit : s);
+}
+
+// Row data of a query tile staged beside its Q and dO (lse and D
+// head-major, as they lie in memory; each position's routing weights of the
+// key block's chunks and the mask word holding them), and the row table the
+// key threads build from it: per chunk of the block and row t = p G + h of
+// the tile, the exponent offset (log2 units: routing bias minus lse; -inf
+// where the row does not see the chunk) and D.
+template <int NCK>
+struct BwdTile {
+  float lse[128];
+  float D[128];
+  float w[32][2];
+  uint32_t mword[32];
+  float off[NCK][128];
+  float dd[NCK][128];
+};
+
 template <int CHUNK>
-__global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(
+__global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const BwdParams prm) {
   constexpr int D = 128;
   constexpr int KB = 128;                        // keys per CTA
   constexpr int NCK = KB / CHUNK;                // chunks per key block (2 or 1)
-  constexpr int NS = 2;                          // query-tile ring depth
+  constexpr int NS = kBwdDkvStages;
+  constexpr int NKT = 32 * kBwdKeyWarps;         // key threads
+  constexpr int W_PROD = kBwdKeyWarps, W_MMA = kBwdKeyWarps + 1;
   constexpr int QBOX = 128 * 128;                // 128 rows x 128 B
   constexpr int T_BYTES = 2 * QBOX;              // one 128 x 128 bf16 tile
+  // TMEM columns: dK, dV accumulators | S^T (then P^T) | dP^T (then dS^T)
   constexpr uint32_t TM_DK = 0, TM_DV = 128, TM_S = 256, TM_DP = 384;
+  using Tile = BwdTile<NCK>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned by pointer arithmetic on the shared array, so that the
+  // compiler keeps the shared address space (and emits shared loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sK = smem;                            // the block's keys (two 64-column boxes)
   uint8_t* sV = sK + T_BYTES;
   uint8_t* sQ = sV + T_BYTES;                    // [NS] query tiles
   uint8_t* sdO = sQ + NS * T_BYTES;              // [NS]
-  BwdRowInfo* info = reinterpret_cast<BwdRowInfo*>(sdO + NS * T_BYTES);   // [NS]
-  float2* rowtab = reinterpret_cast<float2*>(info + NS);                  // [2][NCK][128]
+  Tile* tiles = reinterpret_cast<Tile*>(sdO + NS * T_BYTES);   // [NS]
 
-  __shared__ __align__(8) uint64_t bar_kv, bar_full[NS], bar_empty[NS], bar_st_full, bar_p_full, bar_fin;
+  // Q (with the row data) and dO have rings of their own: dV(n) is the last
+  // reader of dO(n), dK(n) of Q(n), half a tile later
+  __shared__ __align__(8) uint64_t bar_kv, bar_full[NS], bar_empty[NS], bar_full_do[NS], bar_empty_do[NS];
+  __shared__ __align__(8) uint64_t bar_s_full, bar_dp_full, bar_p_full, bar_ds_full, bar_fin;
   __shared__ int slot_tile[NS];
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_s;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_kb = (prm.seq + KB - 1) / KB;      // the grid's key blocks (the last may be half)
-  const int kb = (int)(blockIdx.x % n_kb);       // early key blocks (the most tiles) first
-  const int bg = (int)(blockIdx.x / n_kb);
+  const int split = (int)(blockIdx.x % prm.n_split);
+  const int kb = (int)((blockIdx.x / prm.n_split) % n_kb);   // early key blocks (the most tiles) first
+  const int bg = (int)(blockIdx.x / prm.n_split / n_kb);
   const int b = bg / prm.n_kv, g = bg % prm.n_kv;
   const int P = prm.P, G = prm.G;
   const int kc0 = kb * NCK;                      // first chunk of the key block
   const int key0 = kb * KB;
 
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tmem_alloc(&tmem_slot, 512);
     tmem_relinquish();
   }
@@ -534,9 +618,13 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bar_full[s], 1 + 32);           // TMA bytes + the 32 producer lanes' copies
       mbar_init(&bar_empty[s], 1);
+      mbar_init(&bar_full_do[s], 1);
+      mbar_init(&bar_empty_do[s], 1);
     }
-    mbar_init(&bar_st_full, 1);
-    mbar_init(&bar_p_full, 128);
+    mbar_init(&bar_s_full, 1);
+    mbar_init(&bar_dp_full, 1);
+    mbar_init(&bar_p_full, NKT);
+    mbar_init(&bar_ds_full, NKT);
     mbar_init(&bar_fin, 1);
     abort_s = 0;
     fence_mbar_init();
@@ -546,12 +634,13 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
-  if (warp == 4) {
+  if (warp == W_PROD) {
     // ------------------------------------------------------------ producer
     // K, V of the key block once; then, in position order, every query tile
-    // whose rows attend to a key of the block: the tiles of the block's own
+    // whose rows attend to a key of the block -- the tiles of the block's own
     // chunks (causal) and the later tiles whose routed union (written by the
-    // dQ kernel) holds one of the block's chunks.  A tile id of -1 ends it.
+    // dQ kernel) holds one of the block's chunks -- keeping the ordinals that
+    // fall to this split.  A tile id of -1 ends the walk.
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar_kv, 2 * T_BYTES);
 #pragma unroll
@@ -567,7 +656,9 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(
 #pragma unroll
     for (int ck = 0; ck < NCK; ++ck) bsel |= 1u << ((kc0 + ck) & 31);
     const uint32_t* tm_row = prm.tmask + ((size_t)bg * prm.nw + wsel) * prm.n_tiles;
-    int n_it = 0;                                // tiles issued
+    int n_it = 0;                                // tiles issued (Q and dO)
+    int n_do = 0;                                // tiles whose dO was issued
+    int ord = 0;                                 // relevant tiles seen
     bool go = true;
     for (int t0 = tile0; go && t0 < prm.n_tiles; t0 += 32) {
       const int tt = t0 + lane;
@@ -576,23 +667,32 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(
       while (ballot) {
         const int bit = __ffs(ballot) - 1;
         ballot &= ballot - 1;
+        if (ord++ % prm.n_split != split) continue;
         const int tt2 = t0 + bit;
         const int s = n_it % NS;
+        const int pos_t = tt2 * P;
+        // dO first: its slot is freed half a tile before Q's
         int okw = 1;
+        if (n_it >= NS && lane == 0) okw = (int)mbar_wait(&bar_empty_do[s], ((n_it / NS) - 1) & 1, &abort_s);
+        if (!__shfl_sync(0xffffffffu, okw, 0)) { go = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar_full_do[s], T_BYTES);
+#pragma unroll
+          for (int kb2 = 0; kb2 < 2; ++kb2)
+            tma_load_3d(sdO + s * T_BYTES + kb2 * QBOX, &tmdO, &bar_full_do[s], kb2 * 64, b * prm.n_q + g * G, pos_t);
+        }
+        n_do = n_it + 1;
         if (n_it >= NS && lane == 0) okw = (int)mbar_wait(&bar_empty[s], ((n_it / NS) - 1) & 1, &abort_s);
         if (!__shfl_sync(0xffffffffu, okw, 0)) { go = false; break; }
-        const int pos_t = tt2 * P;
         if (lane == 0) {
           slot_tile[s] = tt2;
-          mbar_arrive_expect_tx(&bar_full[s], 2 * T_BYTES);
+          mbar_arrive_expect_tx(&bar_full[s], T_BYTES);
 #pragma unroll
-          for (int kb2 = 0; kb2 < 2; ++kb2) {
+          for (int kb2 = 0; kb2 < 2; ++kb2)
             tma_load_3d(sQ + s * T_BYTES + kb2 * QBOX, &tmQ, &bar_full[s], kb2 * 64, b * prm.n_q + g * G, pos_t);
-            tma_load_3d(sdO + s * T_BYTES + kb2 * QBOX, &tmdO, &bar_full[s], kb2 * 64, b * prm.n_q + g * G, pos_t);
-          }
         }
         // lse and D: head h's P positions are contiguous (16-byte pieces)
-        BwdRowInfo* in = info + s;
+        Tile* in = tiles + s;
         for (int e = lane; e < 2 * G * (P / 4); e += 32) {
           const int which = e / (G * (P / 4));
           const int rem = e % (G * (P / 4));
@@ -625,12 +725,15 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(
       }
     }
     if (abort_s && lane == 0) {
+      // copies in flight: K, V and the last NS tiles' dO and Q
       mbar_wait(&bar_kv, 0, nullptr);
+      for (int j = (n_do > NS ? n_do - NS : 0); j < n_do; ++j)
+        mbar_wait(&bar_full_do[j % NS], (j / NS) & 1, nullptr);
       for (int j = (n_it > NS ? n_it - NS : 0); j < n_it; ++j)
         mbar_wait(&bar_full[j % NS], (j / NS) & 1, nullptr);
     }
     cp_async_wait_all();
-  } else if (warp == 5) {
+  } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idT = idesc_bf16_f32(128, 128, 0, 0);    // S^T, dP^T: keys x rows
     constexpr uint32_t idA = idesc_bf16_f32(128, D, 0, 1);      // dV, dK: keys x d
@@ -644,191 +747,297 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(
     auto wait_all = [&](uint64_t* bar, uint32_t par) {
       return __all_sync(0xffffffffu, mbar_wait(bar, par, &abort_s));
     };
-    bool ok = wait_all(&bar_kv, 0);
-    for (int n = 0; ok; ++n) {
-      const int s = n % NS;
-      if (!(ok = wait_all(&bar_full[s], (n / NS) & 1))) break;
-      if (slot_tile[s] < 0) break;
-      tc_fence_after();
-      const uint32_t so = (uint32_t)(s * T_BYTES);
+    // S^T(n) or dP^T(n) from ring slot s
+    auto issue_t = [&](uint32_t dst, uint64_t a0, uint64_t b0, int s, uint64_t* bar) {
       if (leader) {
+        const uint32_t so = (uint32_t)(s * T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * QBOX + (kk & 3) * 32;
-          tc_mma_ss(tmem + TM_S, dKk + (off >> 4), dQk0 + ((so + off) >> 4), idT, kk > 0 ? 1u : 0u);
+          tc_mma_ss(dst, a0 + (off >> 4), b0 + ((so + off) >> 4), idT, kk > 0 ? 1u : 0u);
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * QBOX + (kk & 3) * 32;
-          tc_mma_ss(tmem + TM_DP, dVk + (off >> 4), ddOk0 + ((so + off) >> 4), idT, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bar_st_full);
+        tc_commit(bar);
       }
       __syncwarp();
+    };
+    // dV or dK += (P^T or dS^T) (dO or Q): K-steps of 16 rows; rows 64 h +
+    // 16 j .. of the packed operand sit at columns 64 h + 8 j
+    auto issue_a = [&](uint32_t dst, uint32_t a_tm, uint64_t b0, int s, bool first) {
+      if (leader) {
+        const uint32_t so = (uint32_t)(s * T_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          tc_mma_ts(dst, a_tm + (kk >> 2) * 64 + (kk & 3) * 8, b0 + ((so + kk * 2048) >> 4), idA,
+                    (!first || kk > 0) ? 1u : 0u);
+      }
+    };
+    bool ok_do = true;
+    // tile n's Q and row data have landed; false at the end of the walk or on
+    // a timeout
+    auto next_tile = [&](int n, bool& ok) {
+      const int s = n % NS;
+      if (!(ok = wait_all(&bar_full[s], (n / NS) & 1))) return false;
+      tc_fence_after();
+      return slot_tile[s] >= 0;
+    };
+    // dO of tile n has landed
+    auto wait_do = [&](int n) {
+      if (!(ok_do = wait_all(&bar_full_do[n % NS], (n / NS) & 1))) return false;
+      tc_fence_after();
+      return true;
+    };
+    bool ok = wait_all(&bar_kv, 0);
+    bool have = ok && next_tile(0, ok);
+    if (have) {
+      issue_t(tmem + TM_S, dKk, dQk0, 0, &bar_s_full);
+      if (wait_do(0)) issue_t(tmem + TM_DP, dVk, ddOk0, 0, &bar_dp_full);
+      else have = ok = false;
+    }
+    for (int n = 0; have; ++n) {
+      const int s = n % NS;
       if (!(ok = wait_all(&bar_p_full, n & 1))) break;
       tc_fence_after();
-      if (leader) {
-        // dV += P^T dO, dK += dS^T Q: K-steps of 16 query rows
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          tc_mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8, ddOm0 + ((so + kk * 2048) >> 4), idA,
-                    (n > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          tc_mma_ts(tmem + TM_DK, tmem + TM_DP + kk * 8, dQm0 + ((so + kk * 2048) >> 4), idA,
-                    (n > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&bar_empty[s]);
-      }
+      issue_a(tmem + TM_DV, tmem + TM_S, ddOm0, s, n == 0);
+      if (leader) tc_commit(&bar_empty_do[s]);
       __syncwarp();
+      have = next_tile(n + 1, ok);
+      if (!ok) break;
+      if (have) issue_t(tmem + TM_S, dKk, dQk0, (n + 1) % NS, &bar_s_full);
+      if (!(ok = wait_all(&bar_ds_full, n & 1))) break;
+      tc_fence_after();
+      issue_a(tmem + TM_DK, tmem + TM_DP, dQm0, s, n == 0);
+      if (leader) tc_commit(&bar_empty[s]);
+      __syncwarp();
+      if (have) {
+        if (!wait_do(n + 1)) {
+          ok = false;
+          break;
+        }
+        issue_t(tmem + TM_DP, dVk, ddOk0, (n + 1) % NS, &bar_dp_full);
+      }
     }
     if (leader) tc_commit(&bar_fin);
     __syncwarp();
     if (abort_s && lane == 0) mbar_wait(&bar_fin, 0, nullptr);
   } else {
-    // ------------------------------------------------------------ key threads (warps 0-3)
-    const int k = tid;                           // key of the block = TMEM lane
+    // ------------------------------------------------------------ key threads (warps 0-7)
+    const int k = tid & 127;                     // key of the block = TMEM lane
+    const int half = warp >> 2;                  // rows 64 half .. 64 half + 63 of a tile
     const int kpos = key0 + k;
     const int kchunk = kpos / CHUNK;
     const int ck = kchunk - kc0;                 // the key's chunk within the block
     const uint32_t tlane = (uint32_t)((warp & 3) * 32) << 16;
-    const float scale = prm.scale_log2;
-    bool ok = mbar_wait(&bar_kv, 0, &abort_s);
+    const uint64_t sc2 = f2_pack(prm.scale_log2, prm.scale_log2);
+    bool ok = true;
     int n = 0;
     for (;; ++n) {
-      // every exit of this loop is taken by all 128 key threads together: the
+      // every exit of this loop is taken by all key threads together: the
       // named barrier below is reached once per tile by each of them
       const int s = n % NS;
       const bool okw = ok && mbar_wait(&bar_full[s], (n / NS) & 1, &abort_s);
       const int tt = okw ? slot_tile[s] : -1;
-      const BwdRowInfo* in = info + s;
+      Tile* in = tiles + s;
       const int pos_t = tt * P;
       const int c_t = pos_t / CHUNK;
-      // row table of the tile (row t = p G + h): per chunk of the block the
-      // exponent offset (log2 units: routing bias minus lse; -inf where the
-      // row does not see the chunk) and D
-      float2* tab = rowtab + (n & 1) * NCK * 128;
-      if (tt >= 0) {
-        const int t = tid, pp = t >> prm.lgG, hh = t & (G - 1);
+      if (tt >= 0 && (tid >> 7) < NCK) {         // one row-table entry per thread
+        const int c2 = tid >> 7, t = tid & 127;
+        const int pp = t >> prm.lgG, hh = t & (G - 1);
         const int ri = hh * P + pp;
         const float l2 = in->lse[ri] * 1.4426950408889634f;
-        const float Dv = in->D[ri];
-#pragma unroll
-        for (int c2 = 0; c2 < NCK; ++c2) {
-          const int kch = kc0 + c2;
-          float off = -INFINITY;
-          if (kch == c_t) off = -l2;
-          else if (kch < c_t && ((in->mword[pp] >> (kch & 31)) & 1u))
-            off = (prm.sigma != 0.f ? prm.sigma * lg2f(in->w[pp][c2]) : 0.f) - l2;
-          tab[c2 * 128 + t] = make_float2(off, Dv);
-        }
+        const int kch = kc0 + c2;
+        float off = -INFINITY;
+        if (kch == c_t) off = -l2;
+        else if (kch < c_t && ((in->mword[pp] >> (kch & 31)) & 1u))
+          off = (prm.sigma != 0.f ? prm.sigma * lg2f(in->w[pp][c2]) : 0.f) - l2;
+        in->off[c2][t] = off;
+        in->dd[c2][t] = in->D[ri];
       }
-      if (!bar_and_128(1, okw)) { ok = false; break; }
+      if (!bar_and(1, NKT, okw)) { ok = false; break; }
       if (tt < 0) break;                         // uniform once every wait succeeded
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_st_full, n & 1, &abort_s))) {
-        ok = false;                              // the next vote ends the walk
-        continue;
-      }
-      tc_fence_after();
       // causal on the diagonal chunk: row t sees key kpos iff its position
       // pos_t + t / G >= kpos, i.e. t >= (kpos - pos_t) G
       const int colmin = kchunk == c_t ? (kpos - pos_t) * G : 0;
-      const float2* tk = tab + ck * 128;
-#pragma unroll 1
-      for (int q = 0; q < 128 / 32; ++q) {
-        float sv[32], dp[32];
-        tmem_ld32(tmem + tlane + TM_S + q * 32, sv);
-        tmem_ld32(tmem + tlane + TM_DP + q * 32, dp);
-        uint32_t pk[16], dk[16];
+      const float* toff = in->off[ck] + half * 64;
+      const float* tdd = in->dd[ck] + half * 64;
+      const int cm = colmin - half * 64;         // in this warp's columns
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_s_full, n & 1, &abort_s))) {
+        ok = false;
+        continue;                                // the next vote ends the walk
+      }
+      tc_fence_after();
+      float pf[64];                              // P of this key and the warp's 64 rows
+      {
+        float sv[64];
+        tmem_ld64(tmem + tlane + TM_S + half * 64, sv);
+        // p = 2^(s * scale + off): 3 of every 8 pairs on the FMA pipe
+        // (exp2_poly2), the rest on the special-function unit
+        constexpr uint32_t kPolyPairs = 0x52u;   // pairs 1, 4, 6 of each 8
+        uint32_t pk[32];
 #pragma unroll
-        for (int i2 = 0; i2 < 16; ++i2) {
-          float pv[2], dv2[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = q * 32 + 2 * i2 + u;
-            const float2 od = tk[col];
-            const float pr = col >= colmin ? ex2f(fmaf(sv[2 * i2 + u], scale, od.x)) : 0.f;
-            pv[u] = pr;
-            dv2[u] = pr * (dp[2 * i2 + u] - od.y);
+        for (int j = 0; j < 32; ++j) {
+          const float2 o2 = *reinterpret_cast<const float2*>(toff + 2 * j);
+          const uint64_t x = f2_fma(f2_pack(sv[2 * j], sv[2 * j + 1]), sc2, f2_pack(o2.x, o2.y));
+          float e0, e1;
+          if ((kPolyPairs >> (j & 7)) & 1u) {
+            exp2_poly2(x, e0, e1);
+          } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            e0 = ex2f(x0);
+            e1 = ex2f(x1);
           }
-          pk[i2] = pack_bf16x2(pv[0], pv[1]);
-          dk[i2] = pack_bf16x2(dv2[0], dv2[1]);
+          pf[2 * j] = 2 * j >= cm ? e0 : 0.f;
+          pf[2 * j + 1] = 2 * j + 1 >= cm ? e1 : 0.f;
+          pk[j] = pack_bf16x2(pf[2 * j], pf[2 * j + 1]);
         }
-        // P^T over the S^T columns already read, dS^T over dP^T's
-        tmem_st16u(tmem + tlane + TM_S + q * 16, pk);
-        tmem_st16u(tmem + tlane + TM_DP + q * 16, dk);
+        uint32_t h0[16], h1[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          h0[i] = pk[i];
+          h1[i] = pk[16 + i];
+        }
+        tmem_st16u(tmem + tlane + TM_S + half * 64, h0);        // P^T over S^T
+        tmem_st16u(tmem + tlane + TM_S + half * 64 + 16, h1);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_p_full);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_dp_full, n & 1, &abort_s))) {
+        ok = false;
+        continue;
+      }
+      tc_fence_after();
+      {
+        float dp[64];
+        tmem_ld64(tmem + tlane + TM_DP + half * 64, dp);
+        uint32_t h0[16], h1[16];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float2 d2 = *reinterpret_cast<const float2*>(tdd + 2 * j);
+          const uint64_t ds = f2_mul(f2_pack(pf[2 * j], pf[2 * j + 1]),
+                                     f2_sub(f2_pack(dp[2 * j], dp[2 * j + 1]), f2_pack(d2.x, d2.y)));
+          float a0, a1;
+          f2_unpack(ds, a0, a1);
+          (j < 16 ? h0[j] : h1[j - 16]) = pack_bf16x2(a0, a1);
+        }
+        tmem_st16u(tmem + tlane + TM_DP + half * 64, h0);       // dS^T over dP^T
+        tmem_st16u(tmem + tlane + TM_DP + half * 64 + 16, h1);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_ds_full);
     }
-    // kpos < seq is warp-uniform (seq is a multiple of 64)
+    // kpos < seq is warp-uniform (seq is a multiple of 64); warps 0-3 write
+    // dK, warps 4-7 dV
     if (ok && __all_sync(0xffffffffu, mbar_wait(&bar_fin, 0, &abort_s)) && kpos < prm.seq) {
       tc_fence_after();
-      float* krow = prm.dK + ((size_t)bg * prm.seq + kpos) * D;
-      float* vrow = prm.dV + ((size_t)bg * prm.seq + kpos) * D;
+      const bool direct = prm.n_split == 1;
+      const float ks = half ? 1.f : (direct ? prm.scale : 1.f);
+      float* row;
+      if (direct)
+        row = (half ? prm.dV : prm.dK) + ((size_t)bg * prm.seq + kpos) * D;
+      else
+        row = prm.part + (((size_t)split * prm.n_bg + bg) * prm.seq + kpos) * (2 * D) + half * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         float o[32];
         if (n > 0) {
-          tmem_ld32(tmem + tlane + TM_DK + cc * 32, o);
+          tmem_ld32(tmem + tlane + (half ? TM_DV : TM_DK) + cc * 32, o);
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = 0.f;
         }
-        float4* dst = reinterpret_cast<float4*>(krow + cc * 32);
+        float4* dst = reinterpret_cast<float4*>(row + cc * 32);
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4)
-          dst[q4] = make_float4(o[4 * q4] * prm.scale, o[4 * q4 + 1] * prm.scale,
-                                o[4 * q4 + 2] * prm.scale, o[4 * q4 + 3] * prm.scale);
-        if (n > 0) tmem_ld32(tmem + tlane + TM_DV + cc * 32, o);
-        dst = reinterpret_cast<float4*>(vrow + cc * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
+          dst[q4] = make_float4(o[4 * q4] * ks, o[4 * q4 + 1] * ks, o[4 * q4 + 2] * ks, o[4 * q4 + 3] * ks);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
+template <int CHUNK>
 inline size_t attn_bwd_dkv_smem_bytes() {
-  return (size_t)2 * 2 * 128 * 128 + (size_t)2 * 2 * 2 * 128 * 128 + 2 * sizeof(BwdRowInfo) +
-         (size_t)2 * 2 * 128 * sizeof(float2) + 1024;
+  return (size_t)2 * 2 * 128 * 128 + (size_t)kBwdDkvStages * 2 * 2 * 128 * 128 +
+         kBwdDkvStages * sizeof(BwdTile<128 / CHUNK>) + 1024;
 }
 
-// dQ / dw kernel, then the dK / dV kernel, on one stream (the second reads
-// the D rows and tile unions the first writes).  K / V maps: boxes of 64
-// rows (kv64) for the dQ kernel, 128 rows (kv128) for the dK / dV kernel.
+// dK = scale * sum of the splits' partial dK, dV = their sum, in split order.
+__global__ void attn_bwd_dkv_reduce_kernel(const float* __restrict__ part, float* __restrict__ dK,
+                                           float* __restrict__ dV, long long rows, int n_split, float scale) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // one float4 of a row
+  if (i >= rows * 64) return;
+  const long long row = i >> 6;
+  const int c4 = (int)(i & 63);                  // 0..31: dK, 32..63: dV
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < n_split; ++s) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(part + ((size_t)s * rows + row) * 256) + c4);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  if (c4 < 32) {
+    reinterpret_cast<float4*>(dK + row * 128)[c4] =
+        make_float4(acc.x * scale, acc.y * scale, acc.z * scale, acc.w * scale);
+  } else {
+    reinterpret_cast<float4*>(dV + row * 128)[c4 - 32] = acc;
+  }
+}
+
+// dQ / dw kernel, then the dK / dV kernel (and, when the key blocks' tile
+// lists are split, the reduction of the splits), on one stream: each reads
+// what the one before wrote.  K / V maps: boxes of 64 rows (kv64) for the dQ
+// kernel, 128 rows (kv128) for the dK / dV kernel.
 template <int CHUNK>
 cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk64,
                                const CUtensorMap& tv64, const CUtensorMap& tk128,
                                const CUtensorMap& tv128, const BwdParams& prm, cudaStream_t st) {
   const size_t smem_a = attn_bwd_dq_smem_bytes(prm.n_c, prm.nw, prm.P);
-  const size_t smem_b = attn_bwd_dkv_smem_bytes();
+  const size_t smem_b = attn_bwd_dkv_smem_bytes<CHUNK>();
   auto ka = attn_bwd_dq_kernel<CHUNK>;
   auto kb = attn_bwd_dkv_kernel<CHUNK>;
   cudaError_t e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b);
   if (e != cudaSuccess) return e;
-  ka<<<(unsigned)(prm.n_tiles * prm.n_bg), 192, smem_a, st>>>(tq, tdo, tk64, tv64, prm);
+  ka<<<(unsigned)(prm.n_tiles * prm.n_bg), 32 * (kBwdRowWarps + 2), smem_a, st>>>(tq, tdo, tk64, tv64, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int n_kb = (prm.seq + 127) / 128;
-  kb<<<(unsigned)(n_kb * prm.n_bg), 192, smem_b, st>>>(tq, tdo, tk128, tv128, prm);
+  kb<<<(unsigned)(n_kb * prm.n_bg * prm.n_split), 32 * (kBwdKeyWarps + 2), smem_b, st>>>(tq, tdo, tk128, tv128,
+                                                                                   prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || prm.n_split == 1) return e;
+  const long long rows = (long long)prm.n_bg * prm.seq;
+  attn_bwd_dkv_reduce_kernel<<<(unsigned)((rows * 64 + 255) / 256), 256, 0, st>>>(
+      prm.part, prm.dK, prm.dV, rows, prm.n_split, prm.scale);
   return cudaGetLastError();
 }
 
-// Scratch of the two kernels: D rows [b, n_q, seq] fp32 and the tile unions
-// [b * n_kv, nw, seq / P] u32, each 256-byte aligned.
-inline size_t attn_bwd_tc_workspace_bytes(int batch, int n_q, int n_kv, int seq, int n_c) {
+// Scratch of the kernels: D rows [b, n_q, seq] fp32, the tile unions
+// [b * n_kv, nw, seq / P] u32 and, when split, the partial dK | dV rows
+// [n_split, b * n_kv * seq, 256] fp32; each part 256-byte aligned.
+struct BwdWorkspace {
+  size_t d_off, t_off, p_off, total;
+  int n_split;
+};
+
+inline BwdWorkspace attn_bwd_tc_workspace(int batch, int n_q, int n_kv, int seq, int n_c) {
   const int G = n_q / n_kv, P = 128 / G;
-  const size_t d_bytes = ((size_t)batch * n_q * seq * 4 + 255) & ~(size_t)255;
-  const size_t t_bytes = ((size_t)batch * n_kv * ((n_c + 31) / 32) * (seq / P) * 4 + 255) & ~(size_t)255;
-  return d_bytes + t_bytes;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  BwdWorkspace w;
+  w.n_split = attn_bwd_n_split((seq + 127) / 128, batch * n_kv);
+  w.d_off = 0;
+  w.t_off = up((size_t)batch * n_q * seq * 4);
+  w.p_off = w.t_off + up((size_t)batch * n_kv * ((n_c + 31) / 32) * (seq / P) * 4);
+  w.total = w.p_off + (w.n_split > 1 ? up((size_t)w.n_split * batch * n_kv * seq * 256 * 4) : 0);
+  return w;
 }
 
 }  // namespace dash

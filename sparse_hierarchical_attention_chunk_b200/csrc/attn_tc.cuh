@@ -153,8 +153,9 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
   using L = TcLayout<BLK, D>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned by pointer arithmetic on the shared array, so that the
+  // compiler keeps the shared address space (and emits shared loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   int* list = reinterpret_cast<int*>(smem + L::OFF_AUX);             // [n_c + 1]
   uint8_t* code = reinterpret_cast<uint8_t*>(list + prm.n_c + 1);    // [n_c + 1], bit t: tile t active
   uint32_t* mrows = reinterpret_cast<uint32_t*>(

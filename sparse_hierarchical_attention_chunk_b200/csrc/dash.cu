@@ -115,8 +115,8 @@ bool attn_bwd_tc_applies(const dash_problem* p) {
 
 size_t attn_bwd_ws_bytes(const dash_problem* p) {
   if (!attn_bwd_tc_applies(p)) return 0;
-  return dash::attn_bwd_tc_workspace_bytes(p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len,
-                                           n_chunks(p));
+  return dash::attn_bwd_tc_workspace(p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, n_chunks(p))
+      .total;
 }
 
 template <int CHUNK>
@@ -169,9 +169,13 @@ int run_attn_bwd_tc(const dash_problem* p, const void* Q, const void* K, const v
   prm.sigma = p->sigma;
   prm.scale = 1.f / sqrtf((float)d);
   prm.scale_log2 = 1.4426950408889634f * prm.scale;
-  const size_t d_bytes = ((size_t)p->batch * p->n_q_heads * p->seq_len * 4 + 255) & ~(size_t)255;
-  prm.Drow = static_cast<float*>(workspace);
-  prm.tmask = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + d_bytes);
+  const dash::BwdWorkspace ws =
+      dash::attn_bwd_tc_workspace(p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, prm.n_c);
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  prm.Drow = reinterpret_cast<float*>(wsb + ws.d_off);
+  prm.tmask = reinterpret_cast<uint32_t*>(wsb + ws.t_off);
+  prm.part = ws.n_split > 1 ? reinterpret_cast<float*>(wsb + ws.p_off) : nullptr;
+  prm.n_split = ws.n_split;
   if (dw) {
     const cudaError_t e = cudaMemsetAsync(dw, 0, (size_t)prm.n_bg * p->seq_len * prm.n_c * sizeof(float), st);
     if (e != cudaSuccess) return cuda_status(e);

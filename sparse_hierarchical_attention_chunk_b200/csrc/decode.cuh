@@ -566,8 +566,9 @@ __global__ void __launch_bounds__(160, 1) decode_split_kernel(
   constexpr int DT = D / 8;                         // O n-tiles
   constexpr int RS = D + 4;                         // partial row: o[D], m, l, 2 pad (16-B rows)
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned by pointer arithmetic on the shared array, so that the
+  // compiler keeps the shared address space (and emits shared loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   float* red = reinterpret_cast<float*>(smem + NS * STAGE);     // [4 warps][16 rows][RS]
   __shared__ float fac[16][4], rowM[16], rowL[16];
   __shared__ __align__(8) uint64_t full[NS], empty[NS];

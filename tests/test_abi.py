@@ -158,7 +158,13 @@ def test_attn_bwd_workspace_checked(L):
     # for its D rows and tile unions; the reference kernel needs none
     p = _p()
     need = dash.dash_workspace_bytes(p, 2)
-    assert need == 1 * 32 * 1024 * 4 + ((1 * 2 * 1 * (1024 // 8) * 4 + 255) // 256) * 256
+    # D rows [1, 32, 1024] fp32, tile unions [2, 1, 1024 / 8] u32 (256-byte
+    # rounded), and 8 splits of the 16 key blocks' partial dK | dV rows
+    # [8, 2 * 1024, 256] fp32
+    assert need == 1 * 32 * 1024 * 4 + 1024 + 8 * 2 * 1024 * 256 * 4
+    # long sequences have enough key blocks: no split, no partials
+    pl = _p(seq_len=131072, chunk=128)
+    assert dash.dash_workspace_bytes(pl, 2) == 32 * 131072 * 4 + 2 * 32 * (131072 // 8) * 4
     assert dash.dash_workspace_bytes(_p(dtype="f32"), 2) == 0
     assert dash.dash_workspace_bytes(_p(head_dim=64), 2) == 0
     assert dash.dash_workspace_bytes(p, 3) == 0
