@@ -144,6 +144,8 @@ struct TcLayout {
   static_assert(NT * TM_TILE <= TM_COLS, "TMEM budget");
 };
 
+// 320 threads, one CTA per SM: ten warps put three on some of the SM's four
+// sub-partitions, whose 16 K registers then allow 168 per thread.
 template <int CHUNK, int D>
 __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -158,8 +160,8 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc_kernel(
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   int* list = reinterpret_cast<int*>(smem + L::OFF_AUX);             // [n_c + 1]
   uint8_t* code = reinterpret_cast<uint8_t*>(list + prm.n_c + 1);    // [n_c + 1], bit t: tile t active
-  uint32_t* mrows = reinterpret_cast<uint32_t*>(
-      (reinterpret_cast<uintptr_t>(code + prm.n_c + 1) + 15) & ~static_cast<uintptr_t>(15));
+  uint8_t* code_end = code + prm.n_c + 1;                          // rounded up to 16 bytes
+  uint32_t* mrows = reinterpret_cast<uint32_t*>(code_end + ((16u - (smem_u32(code_end) & 15u)) & 15u));
   // compact weights: set bits of each position's mask before each word
   int* mpre = reinterpret_cast<int*>(mrows + 2 * prm.P * prm.nw);          // [2P][nw]
   float* w_sm = reinterpret_cast<float*>(mpre + 2 * prm.P * prm.nw);       // [NS][2P]

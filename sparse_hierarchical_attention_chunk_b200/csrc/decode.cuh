@@ -250,8 +250,7 @@ decode_route_kernel(const __grid_constant__ CUtensorMap tmKb, const DecodeRouteP
   extern __shared__ uint8_t route_smem_raw[];
   // this CTA's slice of the summary cache (TMA, 128-byte swizzle; D / 64
   // boxes of CPC rows x 128 B)
-  uint8_t* sKb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(route_smem_raw) + 1023) &
-                                            ~static_cast<uintptr_t>(1023));
+  uint8_t* sKb = route_smem_raw + ((1024u - (smem_u32(route_smem_raw) & 1023u)) & 1023u);
   __shared__ __align__(8) uint64_t kb_bar[2];   // the two halves of the slice
   // logits of every head for this CTA's chunks (read by the heads' owners
   // after the first cluster barrier), then the staging of p of every head

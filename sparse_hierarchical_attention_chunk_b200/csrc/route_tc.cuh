@@ -86,8 +86,9 @@ __global__ void __launch_bounds__(288, 1) route_tc_kernel(
   constexpr int KT_BOX = KT_ROWS * 128;
   constexpr int KT_BYTES = 2 * KT_BOX;          // one tile, d = 128
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned by pointer arithmetic on the shared array, so that the
+  // compiler keeps the shared address space (and emits shared loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem;
   uint8_t* sKt = smem + Q_BYTES;                // 2 tile slots
   // compact form: once the logits are in TMEM the Kbar tiles are free and
