@@ -529,7 +529,14 @@ def run_ours(args, rank, world, device):
         if rank == 0:
             line["cpu_baseline"] = decode_cpu_baseline(wl, args.cpu_seconds)
         return line
-    main = time_prefill(wl, args.steps, args.warmup, want_clocks=True, keep_routing=rank == 0)
+    if args.backward:
+        entry = time_attn_bwd(wl, args.steps, args.warmup)
+        return {"metric": "stage-2 backward ms (dQ, dK, dV, dw)", "value": entry["bwd_ms"],
+                "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+                "config": workload_config(wl, world), "backward": entry}
+    main = time_prefill(wl, args.steps, args.warmup, want_clocks=True, keep_routing=rank == 0,
+                        packed=args.packed)
     tokens_rank = wl.batch * wl.seq
     value = tokens_rank * world / (main["step_ms"] / 1e3)
     peak = peaks["bf16_tflops"]
@@ -539,7 +546,8 @@ def run_ours(args, rank, world, device):
                 "peak_source": f"{peaks_src} bf16 burst",
                 "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                 "traffic": profile_traffic(
-                    "attn_fwd_tc", wl.name, "sparse_hierarchical_attention_chunk_b200/csrc/attn_tc.cuh"),
+                    "attn_fwd_tc_packed" if args.packed else "attn_fwd_tc", wl.name,
+                    "sparse_hierarchical_attention_chunk_b200/csrc/attn_tc.cuh"),
                 "algorithmic_flops_per_launch": main["flops"],
                 "tile_executed_flops_per_launch": main["exec_flops"],
                 "tile_executed_frac": round(main["exec_flops"] / (main["attn_ms"] / 1e3) / 1e12 / peak, 4),
@@ -626,9 +634,9 @@ def run_ours(args, rank, world, device):
                                  "tile_executed_frac": round(
                                      r["exec_flops"] / (r["attn_ms"] / 1e3) / 1e12 / peak, 4),
                                  "traffic": profile_traffic(
-                                     "attn_fwd_tc", wlx.name,
+                                     "attn_fwd_tc_packed" if packed else "attn_fwd_tc", wlx.name,
                                      "sparse_hierarchical_attention_chunk_b200/csrc/attn_tc.cuh")
-                                 if sigma in (None, wlx.sigma) and not packed else None},
+                                 if sigma in (None, wlx.sigma) else None},
                     "stages": stage_rooflines(r),
                     "support_mean": round(r["support"], 4),
                     "support_per_kv_head": [round(x, 4) for x in r["per_head"]]}
@@ -671,6 +679,7 @@ def run_ours(args, rank, world, device):
         "warmup": args.warmup, "ms_per_step": round(main["step_ms"], 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {**workload_config(wl, world),
+                   "routing_form": "compact (dash_route_packed)" if args.packed else "dense w",
                    "support_mean": round(main["support"], 4),
                    "support_per_kv_head": [round(x, 4) for x in main["per_head"]],
                    "l2": "flushed (256 MiB write) before every timed step"},
@@ -872,6 +881,10 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the 128k prefill / decode lines")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=8.0)
+    ap.add_argument("--packed", action="store_true",
+                    help="main line on the compact routing form (dash_route_packed)")
+    ap.add_argument("--backward", action="store_true",
+                    help="only the stage-2 backward of --workload, beside its forward stage 2")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
