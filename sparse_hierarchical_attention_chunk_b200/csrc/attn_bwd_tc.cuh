@@ -32,6 +32,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <type_traits>
 #include "dash_common.cuh"
 #include "tmem_wide.cuh"
 #include "attn_tc.cuh"
@@ -355,14 +356,20 @@ __global__ void __launch_bounds__(32 * (kBwdRowWarps + 2), 1) attn_bwd_dq_kernel
     // D = dO . O of this row (fp32; each half takes 64 of the d columns), also
     // kept for the key-major kernel
     {
-      float dpp = 0.f;
+      // all sixteen 16-byte loads in flight at once: one round trip
       const uint4* orow = reinterpret_cast<const uint4*>(prm.O + qrow * D + half * 64);
       const uint4* drow = reinterpret_cast<const uint4*>(prm.dO + qrow * D + half * 64);
-#pragma unroll 4
+      uint4 a[8], c[8];
+#pragma unroll
       for (int v = 0; v < 8; ++v) {
-        const uint4 a = __ldg(orow + v), c = __ldg(drow + v);
-        const __nv_bfloat16* xa = reinterpret_cast<const __nv_bfloat16*>(&a);
-        const __nv_bfloat16* xc = reinterpret_cast<const __nv_bfloat16*>(&c);
+        a[v] = __ldg(orow + v);
+        c[v] = __ldg(drow + v);
+      }
+      float dpp = 0.f;
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const __nv_bfloat16* xa = reinterpret_cast<const __nv_bfloat16*>(&a[v]);
+        const __nv_bfloat16* xc = reinterpret_cast<const __nv_bfloat16*>(&c[v]);
 #pragma unroll
         for (int e = 0; e < 8; ++e) dpp = fmaf(__bfloat162float(xa[e]), __bfloat162float(xc[e]), dpp);
       }
@@ -441,26 +448,33 @@ __global__ void __launch_bounds__(32 * (kBwdRowWarps + 2), 1) attn_bwd_dq_kernel
         // (exp2_poly2), the rest on the special-function unit
         constexpr uint32_t kPolyPairs = 0x52u;   // pairs 1, 4, 6 of each 8
         uint32_t pk[16];
+        // the causal test only on the diagonal chunk's blocks
+        auto pass = [&](auto causal) {
 #pragma unroll
-        for (int k2 = 0; k2 < 16; ++k2) {
-          const uint64_t x = f2_fma(f2_pack(sv[2 * k2], sv[2 * k2 + 1]), sc2, off2);
-          float e0, e1;
-          if ((kPolyPairs >> (k2 & 7)) & 1u) {
-            exp2_poly2(x, e0, e1);
-          } else {
-            float x0, x1;
-            f2_unpack(x, x0, x1);
-            e0 = ex2f(x0);
-            e1 = ex2f(x1);
+          for (int k2 = 0; k2 < 16; ++k2) {
+            const uint64_t x = f2_fma(f2_pack(sv[2 * k2], sv[2 * k2 + 1]), sc2, off2);
+            float e0, e1;
+            if ((kPolyPairs >> (k2 & 7)) & 1u) {
+              exp2_poly2(x, e0, e1);
+            } else {
+              float x0, x1;
+              f2_unpack(x, x0, x1);
+              e0 = ex2f(x0);
+              e1 = ex2f(x1);
+            }
+            if (decltype(causal)::value) {
+              e0 = 2 * k2 <= lim ? e0 : 0.f;
+              e1 = 2 * k2 + 1 <= lim ? e1 : 0.f;
+            }
+            const uint64_t d2 = f2_mul(f2_pack(e0, e1), f2_sub(f2_pack(dp[2 * k2], dp[2 * k2 + 1]), D2));
+            float a0, a1;
+            f2_unpack(d2, a0, a1);
+            dsum += a0 + a1;
+            pk[k2] = pack_bf16x2(a0, a1);
           }
-          e0 = 2 * k2 <= lim ? e0 : 0.f;
-          e1 = 2 * k2 + 1 <= lim ? e1 : 0.f;
-          const uint64_t d2 = f2_mul(f2_pack(e0, e1), f2_sub(f2_pack(dp[2 * k2], dp[2 * k2 + 1]), D2));
-          float a0, a1;
-          f2_unpack(d2, a0, a1);
-          dsum += a0 + a1;
-          pk[k2] = pack_bf16x2(a0, a1);
-        }
+        };
+        if (lim < 31) pass(std::true_type{});
+        else pass(std::false_type{});
         tmem_st16u(tb, pk);                    // dS over the half's own S columns
       }
       tmem_wait_st();
@@ -536,7 +550,14 @@ __device__ __forceinline__ bool bar_and(int id, int count, bool v) {
 // dP^T(n + 1), and dS^T(n) while it runs dV(n) and S^T(n + 1).  Eight key
 // warps: two per TMEM lane quarter, each taking 64 of the tile's 128 rows;
 // each keeps its P in registers between the two passes.
-constexpr int kBwdDkvStages = 2;                 // query-tile ring depth
+// Q and dO tiles share one ring of four 32 KB slots.  A tile frees its dO
+// after dV and its Q after dK, half a tile later; the tile two ahead takes
+// the first freed slot for its Q and the second for its dO, so each load
+// has about a whole tile of lead: tile m's Q sits in slot 2 (m & 1) +
+// ((m >> 1) & 1), its dO in the other slot of that pair.
+constexpr int kBwdDkvSlots = 4;
+__device__ __forceinline__ int bwd_qslot(int m) { return 2 * (m & 1) + ((m >> 1) & 1); }
+__device__ __forceinline__ int bwd_dslot(int m) { return 2 * (m & 1) + 1 - ((m >> 1) & 1); }
 constexpr int kBwdKeyWarps = 8;
 // A key block's tile list is split over n_split CTAs (interleaved by tile
 // ordinal) when there are few key blocks: about four waves of 148 SMs.
@@ -573,7 +594,7 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
   constexpr int D = 128;
   constexpr int KB = 128;                        // keys per CTA
   constexpr int NCK = KB / CHUNK;                // chunks per key block (2 or 1)
-  constexpr int NS = kBwdDkvStages;
+  constexpr int NSL = kBwdDkvSlots;
   constexpr int NKT = 32 * kBwdKeyWarps;         // key threads
   constexpr int W_PROD = kBwdKeyWarps, W_MMA = kBwdKeyWarps + 1;
   constexpr int QBOX = 128 * 128;                // 128 rows x 128 B
@@ -587,15 +608,14 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sK = smem;                            // the block's keys (two 64-column boxes)
   uint8_t* sV = sK + T_BYTES;
-  uint8_t* sQ = sV + T_BYTES;                    // [NS] query tiles
-  uint8_t* sdO = sQ + NS * T_BYTES;              // [NS]
-  Tile* tiles = reinterpret_cast<Tile*>(sdO + NS * T_BYTES);   // [NS]
+  uint8_t* sT = sV + T_BYTES;                    // [NSL] Q / dO tile slots
+  Tile* tiles = reinterpret_cast<Tile*>(sT + NSL * T_BYTES);   // [NSL] row data of a Q slot
 
-  // Q (with the row data) and dO have rings of their own: dV(n) is the last
-  // reader of dO(n), dK(n) of Q(n), half a tile later
-  __shared__ __align__(8) uint64_t bar_kv, bar_full[NS], bar_empty[NS], bar_full_do[NS], bar_empty_do[NS];
+  // per slot: filled (TMA bytes plus 32 producer-lane arrivals: the row
+  // data's copies for a Q, plain arrivals for a dO) and freed (by the MMA)
+  __shared__ __align__(8) uint64_t bar_kv, bar_full[NSL], bar_empty[NSL];
   __shared__ __align__(8) uint64_t bar_s_full, bar_dp_full, bar_p_full, bar_ds_full, bar_fin;
-  __shared__ int slot_tile[NS];
+  __shared__ int slot_tile[NSL];                 // the tile whose Q a slot holds
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_s;
 
@@ -615,11 +635,9 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
   }
   if (tid == 0) {
     mbar_init(&bar_kv, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&bar_full[s], 1 + 32);           // TMA bytes + the 32 producer lanes' copies
+    for (int s = 0; s < NSL; ++s) {
+      mbar_init(&bar_full[s], 1 + 32);
       mbar_init(&bar_empty[s], 1);
-      mbar_init(&bar_full_do[s], 1);
-      mbar_init(&bar_empty_do[s], 1);
     }
     mbar_init(&bar_s_full, 1);
     mbar_init(&bar_dp_full, 1);
@@ -656,10 +674,16 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
 #pragma unroll
     for (int ck = 0; ck < NCK; ++ck) bsel |= 1u << ((kc0 + ck) & 31);
     const uint32_t* tm_row = prm.tmask + ((size_t)bg * prm.nw + wsel) * prm.n_tiles;
-    int n_it = 0;                                // tiles issued (Q and dO)
+    int n_it = 0;                                // tiles whose Q was issued
     int n_do = 0;                                // tiles whose dO was issued
     int ord = 0;                                 // relevant tiles seen
     bool go = true;
+    // slot x's fill for tile m: free once its previous use (tile m - 2) is done
+    auto take = [&](int x, int m) {
+      int okw = 1;
+      if (m >= 2 && lane == 0) okw = (int)mbar_wait(&bar_empty[x], ((m >> 1) - 1) & 1, &abort_s);
+      return __shfl_sync(0xffffffffu, okw, 0) != 0;
+    };
     for (int t0 = tile0; go && t0 < prm.n_tiles; t0 += 32) {
       const int tt = t0 + lane;
       const bool rel = tt < prm.n_tiles && (tt < tile_own || (__ldg(tm_row + tt) & bsel) != 0);
@@ -669,30 +693,19 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
         ballot &= ballot - 1;
         if (ord++ % prm.n_split != split) continue;
         const int tt2 = t0 + bit;
-        const int s = n_it % NS;
         const int pos_t = tt2 * P;
-        // dO first: its slot is freed half a tile before Q's
-        int okw = 1;
-        if (n_it >= NS && lane == 0) okw = (int)mbar_wait(&bar_empty_do[s], ((n_it / NS) - 1) & 1, &abort_s);
-        if (!__shfl_sync(0xffffffffu, okw, 0)) { go = false; break; }
+        const int qs = bwd_qslot(n_it), ds = bwd_dslot(n_it);
+        // Q and the row data (the slot freed first)
+        if (!take(qs, n_it)) { go = false; break; }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&bar_full_do[s], T_BYTES);
+          slot_tile[qs] = tt2;
+          mbar_arrive_expect_tx(&bar_full[qs], T_BYTES);
 #pragma unroll
           for (int kb2 = 0; kb2 < 2; ++kb2)
-            tma_load_3d(sdO + s * T_BYTES + kb2 * QBOX, &tmdO, &bar_full_do[s], kb2 * 64, b * prm.n_q + g * G, pos_t);
-        }
-        n_do = n_it + 1;
-        if (n_it >= NS && lane == 0) okw = (int)mbar_wait(&bar_empty[s], ((n_it / NS) - 1) & 1, &abort_s);
-        if (!__shfl_sync(0xffffffffu, okw, 0)) { go = false; break; }
-        if (lane == 0) {
-          slot_tile[s] = tt2;
-          mbar_arrive_expect_tx(&bar_full[s], T_BYTES);
-#pragma unroll
-          for (int kb2 = 0; kb2 < 2; ++kb2)
-            tma_load_3d(sQ + s * T_BYTES + kb2 * QBOX, &tmQ, &bar_full[s], kb2 * 64, b * prm.n_q + g * G, pos_t);
+            tma_load_3d(sT + qs * T_BYTES + kb2 * QBOX, &tmQ, &bar_full[qs], kb2 * 64, b * prm.n_q + g * G, pos_t);
         }
         // lse and D: head h's P positions are contiguous (16-byte pieces)
-        Tile* in = tiles + s;
+        Tile* in = tiles + qs;
         for (int e = lane; e < 2 * G * (P / 4); e += 32) {
           const int which = e / (G * (P / 4));
           const int rem = e % (G * (P / 4));
@@ -707,30 +720,40 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
         }
         for (int p2 = lane; p2 < P; p2 += 32)
           cp_async_4(&in->mword[p2], prm.mask + ((size_t)bg * prm.seq + pos_t + p2) * prm.nw + wsel);
-        cp_async_arrive_noinc(&bar_full[s]);
-        ++n_it;
+        cp_async_arrive_noinc(&bar_full[qs]);
+        n_it = n_it + 1;
+        // dO
+        if (!take(ds, n_it - 1)) { go = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar_full[ds], T_BYTES);
+#pragma unroll
+          for (int kb2 = 0; kb2 < 2; ++kb2)
+            tma_load_3d(sT + ds * T_BYTES + kb2 * QBOX, &tmdO, &bar_full[ds], kb2 * 64, b * prm.n_q + g * G, pos_t);
+        }
+        __syncwarp();
+        mbar_arrive(&bar_full[ds]);
+        n_do = n_it;
       }
     }
     if (go) {
-      const int s = n_it % NS;
-      int okw = 1;
-      if (n_it >= NS && lane == 0) okw = (int)mbar_wait(&bar_empty[s], ((n_it / NS) - 1) & 1, &abort_s);
-      if (__shfl_sync(0xffffffffu, okw, 0)) {
+      // end of the walk: the next tile's Q slot carries tile id -1
+      const int qs = bwd_qslot(n_it);
+      if (take(qs, n_it)) {
         if (lane == 0) {
-          slot_tile[s] = -1;
-          mbar_arrive(&bar_full[s]);
+          slot_tile[qs] = -1;
+          mbar_arrive(&bar_full[qs]);
         }
         __syncwarp();
-        mbar_arrive(&bar_full[s]);
+        mbar_arrive(&bar_full[qs]);
       }
     }
     if (abort_s && lane == 0) {
-      // copies in flight: K, V and the last NS tiles' dO and Q
+      // copies in flight: K, V and the last two tiles' Q and dO
       mbar_wait(&bar_kv, 0, nullptr);
-      for (int j = (n_do > NS ? n_do - NS : 0); j < n_do; ++j)
-        mbar_wait(&bar_full_do[j % NS], (j / NS) & 1, nullptr);
-      for (int j = (n_it > NS ? n_it - NS : 0); j < n_it; ++j)
-        mbar_wait(&bar_full[j % NS], (j / NS) & 1, nullptr);
+      for (int j = (n_it > 2 ? n_it - 2 : 0); j < n_it; ++j)
+        mbar_wait(&bar_full[bwd_qslot(j)], (j >> 1) & 1, nullptr);
+      for (int j = (n_do > 2 ? n_do - 2 : 0); j < n_do; ++j)
+        mbar_wait(&bar_full[bwd_dslot(j)], (j >> 1) & 1, nullptr);
     }
     cp_async_wait_all();
   } else if (warp == W_MMA) {
@@ -740,10 +763,8 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
     const bool leader = elect_one();
     const uint64_t dKk = sw128_desc(smem_u32(sK), 16, 1024);     // K, V as the K-major A
     const uint64_t dVk = sw128_desc(smem_u32(sV), 16, 1024);
-    const uint64_t dQk0 = sw128_desc(smem_u32(sQ), 16, 1024);    // Q, dO as the K-major B
-    const uint64_t ddOk0 = sw128_desc(smem_u32(sdO), 16, 1024);
-    const uint64_t dQm0 = sw128_desc(smem_u32(sQ), QBOX, 1024);  // Q, dO as the MN-major B
-    const uint64_t ddOm0 = sw128_desc(smem_u32(sdO), QBOX, 1024);
+    const uint64_t dTk0 = sw128_desc(smem_u32(sT), 16, 1024);    // Q, dO as the K-major B
+    const uint64_t dTm0 = sw128_desc(smem_u32(sT), QBOX, 1024);  // Q, dO as the MN-major B
     auto wait_all = [&](uint64_t* bar, uint32_t par) {
       return __all_sync(0xffffffffu, mbar_wait(bar, par, &abort_s));
     };
@@ -771,49 +792,47 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
                     (!first || kk > 0) ? 1u : 0u);
       }
     };
-    bool ok_do = true;
     // tile n's Q and row data have landed; false at the end of the walk or on
     // a timeout
     auto next_tile = [&](int n, bool& ok) {
-      const int s = n % NS;
-      if (!(ok = wait_all(&bar_full[s], (n / NS) & 1))) return false;
+      const int x = bwd_qslot(n);
+      if (!(ok = wait_all(&bar_full[x], (n >> 1) & 1))) return false;
       tc_fence_after();
-      return slot_tile[s] >= 0;
+      return slot_tile[x] >= 0;
     };
     // dO of tile n has landed
     auto wait_do = [&](int n) {
-      if (!(ok_do = wait_all(&bar_full_do[n % NS], (n / NS) & 1))) return false;
+      if (!wait_all(&bar_full[bwd_dslot(n)], (n >> 1) & 1)) return false;
       tc_fence_after();
       return true;
     };
     bool ok = wait_all(&bar_kv, 0);
     bool have = ok && next_tile(0, ok);
     if (have) {
-      issue_t(tmem + TM_S, dKk, dQk0, 0, &bar_s_full);
-      if (wait_do(0)) issue_t(tmem + TM_DP, dVk, ddOk0, 0, &bar_dp_full);
+      issue_t(tmem + TM_S, dKk, dTk0, bwd_qslot(0), &bar_s_full);
+      if (wait_do(0)) issue_t(tmem + TM_DP, dVk, dTk0, bwd_dslot(0), &bar_dp_full);
       else have = ok = false;
     }
     for (int n = 0; have; ++n) {
-      const int s = n % NS;
       if (!(ok = wait_all(&bar_p_full, n & 1))) break;
       tc_fence_after();
-      issue_a(tmem + TM_DV, tmem + TM_S, ddOm0, s, n == 0);
-      if (leader) tc_commit(&bar_empty_do[s]);
+      issue_a(tmem + TM_DV, tmem + TM_S, dTm0, bwd_dslot(n), n == 0);
+      if (leader) tc_commit(&bar_empty[bwd_dslot(n)]);
       __syncwarp();
       have = next_tile(n + 1, ok);
       if (!ok) break;
-      if (have) issue_t(tmem + TM_S, dKk, dQk0, (n + 1) % NS, &bar_s_full);
+      if (have) issue_t(tmem + TM_S, dKk, dTk0, bwd_qslot(n + 1), &bar_s_full);
       if (!(ok = wait_all(&bar_ds_full, n & 1))) break;
       tc_fence_after();
-      issue_a(tmem + TM_DK, tmem + TM_DP, dQm0, s, n == 0);
-      if (leader) tc_commit(&bar_empty[s]);
+      issue_a(tmem + TM_DK, tmem + TM_DP, dTm0, bwd_qslot(n), n == 0);
+      if (leader) tc_commit(&bar_empty[bwd_qslot(n)]);
       __syncwarp();
       if (have) {
         if (!wait_do(n + 1)) {
           ok = false;
           break;
         }
-        issue_t(tmem + TM_DP, dVk, ddOk0, (n + 1) % NS, &bar_dp_full);
+        issue_t(tmem + TM_DP, dVk, dTk0, bwd_dslot(n + 1), &bar_dp_full);
       }
     }
     if (leader) tc_commit(&bar_fin);
@@ -833,8 +852,8 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
     for (;; ++n) {
       // every exit of this loop is taken by all key threads together: the
       // named barrier below is reached once per tile by each of them
-      const int s = n % NS;
-      const bool okw = ok && mbar_wait(&bar_full[s], (n / NS) & 1, &abort_s);
+      const int s = bwd_qslot(n);
+      const bool okw = ok && mbar_wait(&bar_full[s], (n >> 1) & 1, &abort_s);
       const int tt = okw ? slot_tile[s] : -1;
       Tile* in = tiles + s;
       const int pos_t = tt * P;
@@ -873,23 +892,38 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
         // (exp2_poly2), the rest on the special-function unit
         constexpr uint32_t kPolyPairs = 0x52u;   // pairs 1, 4, 6 of each 8
         uint32_t pk[32];
+        // the causal test only where the tile holds the key's own chunk
+        // (warp-uniform: a warp's 32 keys lie in one chunk)
+        auto pass = [&](auto causal) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float2 o2 = *reinterpret_cast<const float2*>(toff + 2 * j);
-          const uint64_t x = f2_fma(f2_pack(sv[2 * j], sv[2 * j + 1]), sc2, f2_pack(o2.x, o2.y));
-          float e0, e1;
-          if ((kPolyPairs >> (j & 7)) & 1u) {
-            exp2_poly2(x, e0, e1);
-          } else {
-            float x0, x1;
-            f2_unpack(x, x0, x1);
-            e0 = ex2f(x0);
-            e1 = ex2f(x1);
+          for (int j2 = 0; j2 < 16; ++j2) {
+            const float4 o4 = *reinterpret_cast<const float4*>(toff + 4 * j2);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int j = 2 * j2 + h2;
+              const uint64_t x = f2_fma(f2_pack(sv[2 * j], sv[2 * j + 1]), sc2,
+                                        h2 ? f2_pack(o4.z, o4.w) : f2_pack(o4.x, o4.y));
+              float e0, e1;
+              if ((kPolyPairs >> (j & 7)) & 1u) {
+                exp2_poly2(x, e0, e1);
+              } else {
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                e0 = ex2f(x0);
+                e1 = ex2f(x1);
+              }
+              if (decltype(causal)::value) {
+                e0 = 2 * j >= cm ? e0 : 0.f;
+                e1 = 2 * j + 1 >= cm ? e1 : 0.f;
+              }
+              pf[2 * j] = e0;
+              pf[2 * j + 1] = e1;
+              pk[j] = pack_bf16x2(e0, e1);
+            }
           }
-          pf[2 * j] = 2 * j >= cm ? e0 : 0.f;
-          pf[2 * j + 1] = 2 * j + 1 >= cm ? e1 : 0.f;
-          pk[j] = pack_bf16x2(pf[2 * j], pf[2 * j + 1]);
-        }
+        };
+        if (cm > 0) pass(std::true_type{});
+        else pass(std::false_type{});
         uint32_t h0[16], h1[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -912,13 +946,18 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
         tmem_ld64(tmem + tlane + TM_DP + half * 64, dp);
         uint32_t h0[16], h1[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float2 d2 = *reinterpret_cast<const float2*>(tdd + 2 * j);
-          const uint64_t ds = f2_mul(f2_pack(pf[2 * j], pf[2 * j + 1]),
-                                     f2_sub(f2_pack(dp[2 * j], dp[2 * j + 1]), f2_pack(d2.x, d2.y)));
-          float a0, a1;
-          f2_unpack(ds, a0, a1);
-          (j < 16 ? h0[j] : h1[j - 16]) = pack_bf16x2(a0, a1);
+        for (int j2 = 0; j2 < 16; ++j2) {
+          const float4 d4 = *reinterpret_cast<const float4*>(tdd + 4 * j2);
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int j = 2 * j2 + h2;
+            const uint64_t ds = f2_mul(f2_pack(pf[2 * j], pf[2 * j + 1]),
+                                       f2_sub(f2_pack(dp[2 * j], dp[2 * j + 1]),
+                                              h2 ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y)));
+            float a0, a1;
+            f2_unpack(ds, a0, a1);
+            (j < 16 ? h0[j] : h1[j - 16]) = pack_bf16x2(a0, a1);
+          }
         }
         tmem_st16u(tmem + tlane + TM_DP + half * 64, h0);       // dS^T over dP^T
         tmem_st16u(tmem + tlane + TM_DP + half * 64 + 16, h1);
@@ -964,8 +1003,8 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
 
 template <int CHUNK>
 inline size_t attn_bwd_dkv_smem_bytes() {
-  return (size_t)2 * 2 * 128 * 128 + (size_t)kBwdDkvStages * 2 * 2 * 128 * 128 +
-         kBwdDkvStages * sizeof(BwdTile<128 / CHUNK>) + 1024;
+  return (size_t)2 * 2 * 128 * 128 + (size_t)kBwdDkvSlots * 2 * 128 * 128 +
+         kBwdDkvSlots * sizeof(BwdTile<128 / CHUNK>) + 1024;
 }
 
 // dK = scale * sum of the splits' partial dK, dV = their sum, in split order.
