@@ -223,8 +223,10 @@ int dash_attn_fwd(const dash_problem* p, const void* Q, const void* K, const voi
  * bf16 with d = 128 and G in {4, 8, 16} runs on tcgen05 tensor cores: a
  * query-major kernel (dQ, dw; it also writes each row's dO.O and each
  * 128-row tile's routed union to the workspace), then a key-major kernel
- * (dK, dV) over the tiles that attend to each 128 keys; every output
- * element is written once, in a fixed order (no atomics).  Other shapes run
+ * (dK, dV) over the tiles that attend to each 128 keys; when there are few
+ * key blocks (short sequences) their tile lists are split and the splits'
+ * partial dK | dV rows (in the workspace) are summed in split order.  Every
+ * output element is written once, in a fixed order (no atomics).  Other shapes run
  * a reference kernel on CUDA cores that zeroes dK, dV on the stream and
  * accumulates them with atomics (summation order varies from run to run).
  * Errors: NULL or misaligned required pointers, a bad problem ->
