@@ -9,26 +9,29 @@
 //   dp_j = do.v_j,  ds_j = p_j (dp_j - D),
 //   dq = sum_j ds_j k_j / sqrt(d),  dk_j = sum_rows ds_j q / sqrt(d),
 //   dv_j = sum_rows p_j do,  dw_c = sigma / w_c sum_{j in c, group heads} ds_j.
-// Two kernels, neither with atomics (every output element is written by one
-// CTA, in a fixed order):
+// Two kernels, neither with atomics on dQ, dK or dV (every output element is
+// written by one CTA, in a fixed order):
 //
 //   attn_bwd_dq_kernel   query-major, like the forward: one tile of M = 128
 //       rows (P = 128 / G positions x G heads) per CTA walks the diagonal
 //       chunk and the union of its positions' routed chunks in 64-key blocks.
 //       Per block: S = Q K^T and dP = dO V^T (TS-MMAs, Q and dO copied into
-//       TMEM), then the softmax warps form P and dS (written as bf16 over S)
-//       and the row sums of dS (-> dw, summed over the heads of a position by
-//       shuffles), then dQ += dS K (K as the MN-major operand).  S/dP are
-//       double-buffered, so block n+1's S and dP run while block n's dS is
-//       formed.  Also writes D per row, for the key-major kernel.
+//       TMEM), then eight row warps (two per TMEM lane quarter, 32 keys each)
+//       form P and dS (written as bf16 over S) and the row sums of dS (-> dw,
+//       summed over the heads of a position by shuffles; the two halves'
+//       shares added to the zeroed dw), then dQ += dS K (K as the MN-major
+//       operand).  S/dP are double-buffered, so block n+1's S and dP run
+//       while block n's dS is formed.  Also writes D = dO . O per row and each
+//       tile's routed union, for the key-major kernel.
 //   attn_bwd_dkv_kernel  key-major: one CTA per 128 keys (one 128-key chunk
-//       or a pair of 64-key chunks) walks the query tiles whose rows attend to
-//       those keys (the tiles of the keys' own chunks, causal, and every later
-//       tile one of whose positions routes to them, found from the mask).  Per
-//       tile: S^T = K Q^T and dP^T = V dO^T (SS-MMAs, M = 128 keys, N = 128
-//       rows), P^T and dS^T by the key threads (lse, D and the bias of each
-//       row broadcast from shared memory), then dV += P^T dO and
-//       dK += dS^T Q with the accumulators in TMEM for the whole walk.
+//       or a pair of 64-key chunks; with few key blocks, a share of the
+//       block's tiles) walks the query tiles whose rows attend to those keys
+//       (the tiles of the keys' own chunks, causal, and every later tile whose
+//       routed union holds them).  Per tile: S^T = K Q^T and dP^T = V dO^T
+//       (SS-MMAs, M = 128 keys, N = 128 rows), P^T and dS^T by eight key
+//       warps (a row table of exponent offsets and D in shared memory), then
+//       dV += P^T dO and dK += dS^T Q with the accumulators in TMEM for the
+//       whole walk; the next tile's S^T and dP^T are interleaved with them.
 #pragma once
 
 #include <cuda.h>
