@@ -690,13 +690,28 @@ __global__ void __launch_bounds__(32 * (kBwdKeyWarps + 2), 1) attn_bwd_dkv_kerne
     for (int t0 = tile0; go && t0 < prm.n_tiles; t0 += 32) {
       const int tt = t0 + lane;
       const bool rel = tt < prm.n_tiles && (tt < tile_own || (__ldg(tm_row + tt) & bsel) != 0);
-      uint32_t ballot = __ballot_sync(0xffffffffu, rel);
+      // this split's share of the window's relevant tiles
+      uint32_t ballot = __ballot_sync(0xffffffffu, rel), mine = 0u;
       while (ballot) {
         const int bit = __ffs(ballot) - 1;
         ballot &= ballot - 1;
-        if (ord++ % prm.n_split != split) continue;
+        if (ord++ % prm.n_split == split) mine |= 1u << bit;
+      }
+      while (mine) {
+        const int bit = __ffs(mine) - 1;
+        mine &= mine - 1;
         const int tt2 = t0 + bit;
         const int pos_t = tt2 * P;
+        // the next tile of the window into L2 while this one is loaded: a
+        // box with one sector to fetch from DRAM would wait a DRAM round trip
+        if (mine && lane == 0) {
+          const int pn = (t0 + __ffs(mine) - 1) * P;
+#pragma unroll
+          for (int kb2 = 0; kb2 < 2; ++kb2) {
+            tma_prefetch_l2_3d(&tmQ, kb2 * 64, b * prm.n_q + g * G, pn);
+            tma_prefetch_l2_3d(&tmdO, kb2 * 64, b * prm.n_q + g * G, pn);
+          }
+        }
         const int qs = bwd_qslot(n_it), ds = bwd_dslot(n_it);
         // Q and the row data (the slot freed first)
         if (!take(qs, n_it)) { go = false; break; }

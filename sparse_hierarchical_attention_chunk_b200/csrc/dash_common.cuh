@@ -157,6 +157,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
       : "memory");
 }
 
+// Bring a box of a tensor into L2 ahead of its load (no shared memory, no
+// completion to wait for: a hint).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 // The same with an L2 cache policy (from l2_evict_first_policy() and the
 // like) attached to the copy.
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, uint64_t* bar,
