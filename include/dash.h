@@ -415,6 +415,17 @@ int dash_selftest_wait_timeout(void* stream);
  */
 int dash_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
 
+/*
+ * Test hook (no counterpart in the pages): the number of CTAs the
+ * tensor-core dash_attn_bwd splits each key block's tile list over, for
+ * every later call in this process (n = 1 .. 8), or the automatic choice
+ * (n = 0: split only when there are fewer key blocks than about four waves
+ * of SMs).  dash_workspace_bytes(p, 2) follows the setting.  Not thread-safe:
+ * for tests that reach both the split and the unsplit path on small inputs.
+ * Returns the previous setting, or -1 (nothing changed) for n outside 0 .. 8.
+ */
+int dash_selftest_bwd_split(int n);
+
 #ifdef __cplusplus
 }
 #endif

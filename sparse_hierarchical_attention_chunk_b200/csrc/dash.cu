@@ -635,6 +635,13 @@ int dash_selftest_wait_timeout(void* stream) {
   return cuda_status(cudaGetLastError());
 }
 
+int dash_selftest_bwd_split(int n) {
+  if (n < 0 || n > dash::kBwdMaxSplit) return -1;
+  const int prev = dash::attn_bwd_split_setting();
+  dash::attn_bwd_split_setting() = n;
+  return prev;
+}
+
 int dash_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
   if (n < 0 || (n > 0 && (!x || !y))) return DASH_ERR_INVALID_ARG;
   if (n == 0) return DASH_OK;

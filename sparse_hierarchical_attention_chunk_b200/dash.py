@@ -32,7 +32,8 @@ EXPORTED = ("dash_status_str", "dash_version", "dash_summarize", "dash_route", "
             "dash_workspace_bytes", "dash_decode", "dash_decode_varlen", "dash_decode_paged",
             "dash_get_error", "dash_decode_noalloc", "dash_summarize_append", "dash_route_topk",
             "dash_attn_bwd", "dash_route_bwd", "dash_summarize_bwd", "dash_selftest_wait_timeout",
-            "dash_selftest_exp2_poly", "dash_route_packed", "dash_attn_fwd_packed")
+            "dash_selftest_exp2_poly", "dash_route_packed", "dash_attn_fwd_packed",
+            "dash_selftest_bwd_split")
 
 
 class DashError(RuntimeError):
@@ -107,6 +108,8 @@ def lib():
         L.dash_selftest_wait_timeout.argtypes = [vp]
         L.dash_selftest_exp2_poly.restype = i32
         L.dash_selftest_exp2_poly.argtypes = [vp, vp, i32, vp]
+        L.dash_selftest_bwd_split.restype = i32
+        L.dash_selftest_bwd_split.argtypes = [i32]
         L.dash_get_error.restype = i32
         L.dash_get_error.argtypes = [vp]
         L.dash_decode_noalloc.restype = i32
@@ -471,6 +474,15 @@ def dash_selftest_exp2_poly(x, y, stream=None):
     _check(y, "y", (x.numel(),), torch.float32)
     _raise("dash_selftest_exp2_poly",
            lib().dash_selftest_exp2_poly(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)))
+
+
+def dash_selftest_bwd_split(n):
+    """Force the tensor-core backward's split count (1..8; 0 = automatic) for
+    later calls; returns the previous setting (a test hook)."""
+    prev = int(lib().dash_selftest_bwd_split(int(n)))
+    if prev < 0:
+        raise ValueError(f"split count {n} outside 0..8")
+    return prev
 
 
 def dash_get_error(stream=None):

@@ -215,3 +215,20 @@ def test_estimate_diagonal_arguments_checked(L):
                          FAKE, need, None) == dash.DASH_ERR_INVALID_ARG
     assert L.dash_decode_noalloc(ctypes.byref(pd), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
                                  None) == dash.DASH_ERR_UNSUPPORTED
+
+
+def test_bwd_split_hook_sets_the_workspace(L):
+    # the forced split count of the tensor-core backward: no partial rows when
+    # unsplit, n_split of them otherwise; 0 restores the automatic choice
+    p = _p()
+    base = 1 * 32 * 1024 * 4 + 1024
+    rows = 2 * 1024 * 256 * 4
+    try:
+        assert dash.dash_selftest_bwd_split(1) == 0
+        assert dash.dash_workspace_bytes(p, 2) == base
+        assert dash.dash_selftest_bwd_split(3) == 1
+        assert dash.dash_workspace_bytes(p, 2) == base + 3 * rows
+    finally:
+        assert dash.dash_selftest_bwd_split(0) == 3
+    assert dash.dash_workspace_bytes(p, 2) == base + 8 * rows
+    assert L.dash_selftest_bwd_split(9) == -1 and L.dash_selftest_bwd_split(-1) == -1

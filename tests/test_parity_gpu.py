@@ -941,6 +941,35 @@ def test_attn_bwd_matches_oracle(name):
     assert not np64(dw)[~act].any()
 
 
+@pytest.mark.parametrize("split", [1, 3])
+def test_attn_bwd_tc_split_counts(split):
+    # the key-major kernel with each key block's tiles in one CTA (dK, dV
+    # written directly, as for long sequences) and split over three (partial
+    # rows summed by the reduction), on the same inputs as the oracle
+    from oracle import dash_oracle_bwd as obwd
+    wl = BWD["g16_d128_b64_nc37"][0]
+    inp = synth.make_prefill(wl, seed=26)
+    p = dash.problem_for(wl)
+    dev = {n: inp[n].cuda() for n in ("Q", "K", "V", "qbar")}
+    out = dash.prefill(p, dev["Q"], dev["K"], dev["V"], dev["qbar"])
+    dO = torch.randn(dev["Q"].shape, generator=torch.Generator().manual_seed(27)).to(torch.bfloat16)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    g = [torch.full(dev["Q"].shape, 5.0, **f32), torch.full(dev["K"].shape, 5.0, **f32),
+         torch.full(dev["V"].shape, 5.0, **f32), torch.full(out["w"].shape, 5.0, **f32)]
+    prev = dash.dash_selftest_bwd_split(split)
+    try:
+        dash.dash_attn_bwd(p, dev["Q"], dev["K"], dev["V"], out["w"], out["mask"], out["O"],
+                           out["lse"], dO.cuda(), *g)
+        assert dash.dash_get_error() == dash.DASH_OK
+    finally:
+        dash.dash_selftest_bwd_split(prev)
+    ref = obwd.attn_bwd(inp["Q"], inp["K"], inp["V"], np64(out["w"]), mask_from_dev(out["mask"]),
+                        wl.sigma, wl.chunk, dO)
+    for got, want, nm in zip(g, ref, ("dQ", "dK", "dV", "dw")):
+        err = np.abs(np64(got) - want).max() / max(np.abs(want).max(), 1e-30)
+        assert err <= 2e-2, (nm, split, err)
+
+
 def test_attn_bwd_tc_is_deterministic():
     # every output element is written once, in a fixed order: two calls agree bit for bit
     wl = BWD["g16_d128_b64_nc37"][0]
