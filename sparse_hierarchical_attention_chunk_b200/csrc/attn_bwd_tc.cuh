@@ -567,14 +567,7 @@ constexpr int kBwdKeyWarps = 8;
 constexpr int kBwdSplitTarget = 4 * 148;
 constexpr int kBwdMaxSplit = 8;
 
-// 0: automatic; 1 .. kBwdMaxSplit: forced (a test hook)
-inline int& attn_bwd_split_setting() {
-  static int setting = 0;
-  return setting;
-}
-
 inline int attn_bwd_n_split(int n_kb, int n_bg) {
-  if (attn_bwd_split_setting() > 0) return attn_bwd_split_setting();
   const int units = n_kb * n_bg;
   int s = (kBwdSplitTarget + units - 1) / units;
   return s < 1 ? 1 : (s > kBwdMaxSplit ? kBwdMaxSplit : s);

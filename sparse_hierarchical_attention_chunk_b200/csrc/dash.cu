@@ -113,10 +113,24 @@ bool attn_bwd_tc_applies(const dash_problem* p) {
   return p->dtype == DASH_BF16 && p->head_dim == 128 && (G == 4 || G == 8 || G == 16);
 }
 
+// The split count a test forced with dash_selftest_bwd_split (0: automatic).
+int g_bwd_split_forced = 0;
+
+// The backward's workspace layout, with a forced split count applied.
+dash::BwdWorkspace bwd_workspace(const dash_problem* p) {
+  dash::BwdWorkspace ws =
+      dash::attn_bwd_tc_workspace(p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, n_chunks(p));
+  if (g_bwd_split_forced > 0) {
+    ws.n_split = g_bwd_split_forced;
+    const size_t part = (size_t)ws.n_split * p->batch * p->n_kv_heads * p->seq_len * 256 * 4;
+    ws.total = ws.p_off + (ws.n_split > 1 ? ((part + 255) & ~(size_t)255) : 0);
+  }
+  return ws;
+}
+
 size_t attn_bwd_ws_bytes(const dash_problem* p) {
   if (!attn_bwd_tc_applies(p)) return 0;
-  return dash::attn_bwd_tc_workspace(p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, n_chunks(p))
-      .total;
+  return bwd_workspace(p).total;
 }
 
 template <int CHUNK>
@@ -169,8 +183,7 @@ int run_attn_bwd_tc(const dash_problem* p, const void* Q, const void* K, const v
   prm.sigma = p->sigma;
   prm.scale = 1.f / sqrtf((float)d);
   prm.scale_log2 = 1.4426950408889634f * prm.scale;
-  const dash::BwdWorkspace ws =
-      dash::attn_bwd_tc_workspace(p->batch, p->n_q_heads, p->n_kv_heads, p->seq_len, prm.n_c);
+  const dash::BwdWorkspace ws = bwd_workspace(p);
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   prm.Drow = reinterpret_cast<float*>(wsb + ws.d_off);
   prm.tmask = reinterpret_cast<uint32_t*>(wsb + ws.t_off);
@@ -637,8 +650,8 @@ int dash_selftest_wait_timeout(void* stream) {
 
 int dash_selftest_bwd_split(int n) {
   if (n < 0 || n > dash::kBwdMaxSplit) return -1;
-  const int prev = dash::attn_bwd_split_setting();
-  dash::attn_bwd_split_setting() = n;
+  const int prev = g_bwd_split_forced;
+  g_bwd_split_forced = n;
   return prev;
 }
 
