@@ -1,8 +1,11 @@
 """Host-side pieces of bench.py (no GPU): the algorithmic byte count of a
-decode step and the workload config that both arms of the bench print."""
+decode step, the workload config that both arms of the bench print, and the
+DRAM traffic it takes from the committed ncu summaries."""
 
 import importlib.util
 import os
+import re
+import shutil
 
 import torch
 
@@ -55,3 +58,41 @@ def test_workload_config_is_shared_by_both_arms():
         assert ("cache_len" in cfg) == (wl.kind == "decode")
         assert ("cache_lens" in cfg) == (wl.min_len_frac > 0)
         assert ("kv_layout" in cfg) == wl.paged
+
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = "sparse_hierarchical_attention_chunk_b200/csrc/"
+PROFILED = [("attn_fwd_tc", "prefill_bf16_s32768", "attn_tc.cuh"),
+            ("attn_fwd_tc", "prefill_bf16_s131072", "attn_tc.cuh"),
+            ("attn_fwd_tc_packed", "prefill_bf16_s131072", "attn_tc.cuh"),
+            ("decode", "decode_bf16_b8_L131072", "decode.cuh"),
+            ("decode", "decode_varlen_bf16_b8_L131072", "decode.cuh"),
+            ("decode", "decode_paged_bf16_b8_L131072", "decode.cuh")]
+
+
+def _dram_bytes(text):
+    unit = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    return sum(float(v) * unit[u] for v, u in re.findall(r"DRAM (?:read|write)\s+([0-9.]+) (\w+)", text))
+
+
+def test_profile_traffic_of_the_committed_summaries():
+    # every summary the bench line draws on was taken on the current source,
+    # and the traffic it reports is the summary's DRAM read + write
+    for tag, wl, src in PROFILED:
+        got = bench.profile_traffic(tag, wl, CSRC + src)
+        assert got is not None, (tag, wl)
+        text = open(os.path.join(ROOT, "profiles", f"{tag}_{wl}.txt")).read()
+        assert got == int(_dram_bytes(text)), (tag, wl)
+        assert got > 0
+
+
+def test_profile_traffic_is_none_once_the_source_changed(tmp_path, monkeypatch):
+    (tmp_path / "profiles").mkdir()
+    shutil.copy(os.path.join(ROOT, "profiles", "attn_fwd_tc_prefill_bf16_s32768.txt"), tmp_path / "profiles")
+    src = tmp_path / "attn_tc.cuh"
+    src.write_bytes(open(os.path.join(ROOT, CSRC, "attn_tc.cuh"), "rb").read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profile_traffic("attn_fwd_tc", "prefill_bf16_s32768", "attn_tc.cuh") is not None
+    src.write_bytes(src.read_bytes() + b"\n// changed\n")
+    assert bench.profile_traffic("attn_fwd_tc", "prefill_bf16_s32768", "attn_tc.cuh") is None
+    assert bench.profile_traffic("attn_fwd_tc", "no_such_workload", "attn_tc.cuh") is None
